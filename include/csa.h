@@ -1,0 +1,207 @@
+/*
+ * csa.h -- C ABI of libcsa.so: one decode step of combined sparse attention
+ * (pinned prefix + sliding window + Quest-style top-k pages) for the
+ * full-attention layers of hybrid LLMs, over a full-size paged bf16 GQA KV
+ * cache, on NVIDIA B200 (sm_100a).
+ *
+ * What the operation is ("Accelerating Long-Context Decoding in Large-Scale
+ * Hybrid LLMs Without Retraining", abstract; arxivlens analysis of the same
+ * paper, "Methodology"; roboaidigest post, "The Move" and "Why It Matters"):
+ * each query head of a full-attention layer attends to the union of
+ *   - a pinned prefix: the first `prefix` tokens,
+ *   - a sliding window: the last `window` tokens,
+ *   - a fixed budget of the most relevant tokens, chosen query-aware as the
+ *     top-k pages by the Quest upper-bound score
+ *         s_h(p) = sum_i max(q_{h,i} * max_{p,i}, q_{h,i} * min_{p,i})
+ *     where min/max are the per-page, per-channel key extremes,
+ * and the KV cache itself stays full size, so any page can be selected.
+ * Window and budget are per-layer arguments.
+ *
+ * Readings this library takes where the pages are silent:
+ *   - page size is 16 tokens; k = floor(budget_tokens / 16) pages;
+ *   - prefix and window are counted in tokens and applied token-exactly;
+ *     a page is a top-k candidate unless all its valid tokens already lie in
+ *     prefix or window; a selected page contributes all its valid tokens;
+ *   - the score of a kv-head's page is the max over the G query heads of
+ *     the group of the per-head bound (an upper bound for every head);
+ *   - equal scores: the lower logical page index wins; the selected pages
+ *     are returned in ascending page order;
+ *   - softmax scale defaults to 1/sqrt(D); no soft-cap; q and k are taken
+ *     after any positional encoding;
+ *   - scores are unscaled (q.k, not q.k/sqrt(D)); the order is the same.
+ *
+ * ---------------------------------------------------------------- layouts
+ * All tensors are row-major and contiguous; bf16 is IEEE bfloat16.
+ *   q          bf16  [B][Hq][D]                 query of the step
+ *   k_cache    bf16  [num_pages][Hkv][16][D]    keys, one page of one kv-head
+ *   v_cache    bf16  [num_pages][Hkv][16][D]    is a contiguous 32*D-byte tile
+ *   meta       bf16  [num_pages][Hkv][2][D]     row 0 = min, row 1 = max key
+ *   page_table int32 [B][max_pages_per_seq]     logical page -> physical page
+ *   seq_lens   int32 [B]                        valid tokens incl. this step's
+ *   sel_pages  int32 [B][Hkv][max_sel]          selected logical pages
+ *   n_sel      int32 [B][Hkv]
+ *   out        bf16  [B][Hq][D]
+ *   lse        fp32  [B][Hq]                    natural-log sum-exp of scale*q.k
+ * Query head h reads kv-head h / (Hq/Hkv).  Token t of sequence b lives in
+ * physical page page_table[b][t/16], slot t%16.
+ *
+ * ----------------------------------------------------------- conventions
+ *  - Every pointer argument except the ones marked "host" is a DEVICE
+ *    pointer owned by the caller; the library allocates no memory and holds
+ *    no per-call state outside the caller's workspace.
+ *  - Device pointers must be 16-byte aligned (CSA_ERR_INVALID_ARG if not).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All calls
+ *    are asynchronous on it; the status code reports argument checks and
+ *    launch errors only.  Calls sharing one workspace must not overlap.
+ *  - Page ids that fall outside [0, num_pages), selected pages outside the
+ *    candidate range, and a selection that is not strictly ascending are
+ *    detected on the device: the page is skipped and a flag is latched in
+ *    the workspace; csa_get_device_status() reports and clears it.  No
+ *    kernel traps or spins without a bound.
+ *  - Supported shapes: page_size == 16, D in {64, 128, 256},
+ *    Hq/Hkv in {1, 2, 4, 8, 16}, B*Hkv <= 2048; else CSA_ERR_UNSUPPORTED.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = -1, /* null/misaligned pointer, bad size or range  */
+    CSA_ERR_UNSUPPORTED = -2, /* shape outside the supported set             */
+    CSA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required  */
+    CSA_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed        */
+    CSA_ERR_DEVICE_FLAG = -5  /* a kernel latched a device-side error flag   */
+};
+
+/* Bits of the device-side flag word (see csa_get_device_status). */
+enum {
+    CSA_DEVFLAG_BAD_PAGE_ID = 1,  /* page_table entry outside [0, num_pages)  */
+    CSA_DEVFLAG_BAD_SELECTION = 2,/* sel_pages entry outside the candidates,
+                                     not ascending, or n_sel out of range     */
+    CSA_DEVFLAG_BAD_SEQ_LEN = 4,  /* seq_len < 0 or > 16 * max_pages_per_seq,
+                                     or shorter than the appended chunk       */
+    CSA_DEVFLAG_TIMEOUT = 8       /* a bounded pipeline wait gave up          */
+};
+
+/* Problem shape, passed by host pointer to every call. */
+typedef struct csa_dims {
+    int B;                 /* sequences in the batch                          */
+    int Hq;                /* query heads                                     */
+    int Hkv;               /* key/value heads (Hq % Hkv == 0)                 */
+    int D;                 /* head dimension                                  */
+    int page_size;         /* tokens per page; must be 16                     */
+    int max_pages_per_seq; /* row length of page_table                        */
+    int num_pages;         /* physical pages in k_cache / v_cache / meta      */
+    int max_sel;           /* row length of sel_pages (>= budget_tokens / 16) */
+} csa_dims;
+
+/* Bytes of device workspace the calls below need for shape *d (host
+ * pointer).  Returns 0 for an invalid or unsupported shape.  The workspace
+ * holds the device flag word, per-(sequence, kv-head) tickets, the fp32
+ * page scores and the split-K partial results. */
+size_t csa_workspace_size(const csa_dims *d);
+
+/* Zero `bytes` of `workspace` on `stream`.  Required once before the first
+ * call that uses a fresh workspace; the kernels leave their tickets at zero
+ * again when they finish. */
+int csa_workspace_init(void *workspace, size_t bytes, void *stream);
+
+/*
+ * Append tokens to the paged cache and keep the page metadata current
+ * (the full-size cache of "Why It Matters"; the Quest per-page key min/max
+ * used by the top-k selection of "Methodology").
+ *
+ * The last n_new tokens of each sequence, positions [seq_lens[b] - n_new,
+ * seq_lens[b]), are the new ones.  new_k/new_v are bf16 [B][n_new][Hkv][D];
+ * each new token is written to k_cache/v_cache at its page slot.  For every
+ * page that holds a new token, meta is set to the elementwise min/max of
+ * the page's valid keys: from the new keys alone when the page starts within
+ * the new tokens, else from the stored min/max and the new keys (so the
+ * stored metadata of the page's older tokens must be current).
+ * new_k == NULL (and new_v == NULL) is the rebuild mode: nothing is
+ * written to the cache, and meta is recomputed from k_cache for every page
+ * that holds one of positions [max(0, seq_lens[b] - n_new), seq_lens[b]).
+ * seq_lens already include the new tokens.  n_new >= 1 (in rebuild mode any
+ * n_new >= max seq_len rebuilds everything).
+ */
+int csa_meta_update(const csa_dims *d, void *k_cache, void *v_cache, void *meta,
+                    const int32_t *page_table, const int32_t *seq_lens,
+                    const void *new_k, const void *new_v, int n_new,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Query-aware top-k page selection, Quest-style ("Methodology"; "The Move").
+ *
+ * For each (sequence b, kv-head g), with L = seq_lens[b], Pe = min(prefix, L)
+ * and We = min(window, L), the candidates are the logical pages holding at
+ * least one token of [Pe, L - We).  Each candidate gets the fp32 score
+ *   s(p) = max over the G query heads h of group g of
+ *          sum_i max(q_{h,i} * max_{p,i}, q_{h,i} * min_{p,i}),
+ * reading only the page metadata.  The top k' = min(budget_tokens / 16,
+ * #candidates) pages by (score descending, page ascending) are written to
+ * sel_pages[b][g][0..k') in ascending page order and k' to n_sel[b][g].
+ * scores_out (nullable) receives fp32 [B][Hkv][max_pages_per_seq] scores at
+ * the candidate positions (other entries are left untouched).
+ * budget_tokens / 16 must not exceed max_sel.
+ */
+int csa_score_select(const csa_dims *d, const void *q, const void *meta,
+                     const int32_t *page_table, const int32_t *seq_lens,
+                     int prefix, int window, int budget_tokens,
+                     int32_t *sel_pages, int32_t *n_sel, float *scores_out,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Combined sparse attention decode ("Accelerating Long-Context Decoding ...",
+ * abstract): for every query head h of sequence b (kv-head g = h / G),
+ *   A = { t < L : t < Pe  or  t >= L - We  or  page t/16 in sel_pages[b][g] }
+ *   out[b][h] = sum_{t in A} softmax_t(scale * q_h . k_t) v_t
+ *   lse[b][h] = log sum_{t in A} exp(scale * q_h . k_t)
+ * computed split-K across the GPU with an fp32 online softmax; the splits
+ * are merged on the device.  An empty A gives out = 0 and lse = -inf.
+ * sel_pages must be strictly ascending candidate pages (as csa_score_select
+ * writes them).  scale <= 0 selects 1/sqrt(D).  lse is nullable.
+ */
+int csa_decode(const csa_dims *d, const void *q, const void *k_cache, const void *v_cache,
+               const int32_t *page_table, const int32_t *seq_lens,
+               const int32_t *sel_pages, const int32_t *n_sel, int prefix, int window,
+               float scale, void *out, float *lse,
+               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Dense decode over every valid token: the unmodified full-attention layer
+ * the pages compare against ("Results": every configuration is slower than
+ * it at short context).  Same outputs and conventions as csa_decode with
+ * A = { t < L }.
+ */
+int csa_decode_full(const csa_dims *d, const void *q, const void *k_cache,
+                    const void *v_cache, const int32_t *page_table,
+                    const int32_t *seq_lens, float scale, void *out, float *lse,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Synchronise `stream`, read and clear the device flag word of `workspace`.
+ * Returns CSA_OK when no flag was set, CSA_ERR_DEVICE_FLAG when one was (the
+ * CSA_DEVFLAG_* bits go to *flags_out if it is not NULL), CSA_ERR_CUDA on a
+ * CUDA error.
+ */
+int csa_get_device_status(void *workspace, void *stream, int *flags_out);
+
+/* Static string for a status code (host). */
+const char *csa_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int csa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H */
