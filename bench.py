@@ -1,0 +1,508 @@
+#!/usr/bin/env python
+"""Benchmark: combined sparse decode attention, tokens/s per layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload ctx256k|ctx64k]
+
+One step = one decode step of the whole hot path for every layer of the
+workload: append the new token + metadata update, Quest scoring + top-k
+selection, split-K sparse decode + merge.  The default workload is the
+12-layer, batch-4, 262144-token stack (32 query / 4 kv heads, head dim 128,
+prefix 128, per-layer (window, budget) cycling through (512, 1024) ...
+(4096, 8192)); its inputs are synthetic (seeded Gaussian q/K/V in a paged
+cache with a random page permutation).  Each step is one CUDA graph of the
+36 library calls; the K timed steps are replayed back to back between CUDA
+events.  Every layer touches 150-235 MB (1.8-2.8 GB per step), more than the
+126 MB L2, so no flush is needed between steps.
+
+value = tokens/s per layer = B * layers * K / t (whole job: summed over
+ranks, t = max over ranks).  ``roofline`` is measured on the dominant call
+(scoring + selection at 256k) from graph replays over all 12 layers.
+``--impl reference`` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from dataclasses import replace
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from long_context_decoding_b200 import cost  # noqa: E402
+from long_context_decoding_b200 import workloads as wl  # noqa: E402
+
+METRIC = "decode attention tokens/s per layer at 64k/256k ctx, batch 4; % of HBM roofline"
+UNIT = "tokens/s/layer"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=("ctx256k", "ctx64k"), default="ctx256k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the 64k single-layer line")
+    ap.add_argument("--profile", action="store_true",
+                    help="timed steps only (for an ncu launch list): no baseline, e2e, clocks")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- plumbing
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        dev = torch.device("cuda", self.local) if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,utilization.gpu,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        sel = []
+        try:   # nvidia-smi numbers GPUs physically; select ours by UUID
+            sel = ["-i", "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)]
+        except Exception:
+            pass
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "100", *sel],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(", ") for r in self.f.read().strip().splitlines() if r.count(",") >= 9]
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        busy = [r for r in rows if r[3].strip().isdigit() and int(r[3]) >= 50] or rows
+        mhz = [float(r[1]) for r in busy if r[1].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i in range(4) if r[6 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": float(busy[0][2]) if busy[0][2].strip().isdigit() else None,
+                "reasons": reasons, "samples": len(busy)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(w: wl.Workload, seconds: float, steps: int = 0, warmup: int = 0):
+    """Time the CPU oracle on a bounded sample of workload ``w``: one
+    sequence (all its kv-heads and query heads) of the first layer, full
+    length, one decode step (scores -> top-k -> attention) per iteration.
+    Returns (tokens/s per layer, iterations, seconds, threads)."""
+    import oracle
+    threads = oracle.set_threads(len(os.sched_getaffinity(0)))
+    ws = replace(w, B=1, seq_lens=w.seq_lens[:1], layers=1, steps=0, spare_pages=0)
+    c = wl.make_case(ws, "cpu", poison=False)
+    window, budget = w.layer_window_budget(0)
+    d = oracle.Dims(1, ws.Hq, ws.Hkv, ws.D, 16, ws.max_pages, ws.num_pages)
+    h = dict(q=wl.bits(c.q), k=wl.bits(c.k_cache), v=wl.bits(c.v_cache),
+             pt=c.page_table.numpy(), sl=c.seq_lens.numpy())
+    scale = 1.0 / math.sqrt(ws.D)
+
+    def one():
+        oracle.step(d, h["q"], h["k"], h["v"], h["pt"], h["sl"], ws.prefix, window, budget,
+                    max(1, budget // 16), scale)
+
+    for _ in range(warmup):
+        one()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        one()
+        n += 1
+        el = time.perf_counter() - t0
+        if (steps and n >= steps) or (not steps and el >= seconds):
+            break
+    return n / el, n, el, threads, (f"1 of {w.B} sequences of layer 0 (window {window}, budget "
+                                    f"{budget}) at {w.seq_lens[0]} tokens, all {w.Hkv} kv-heads "
+                                    f"and {w.Hq} query heads; one oracle decode step per "
+                                    f"iteration, {n} iterations in {el:.1f} s")
+
+
+def run_reference(args, dist: Dist, w: wl.Workload):
+    if dist.rank != 0:
+        return
+    rate, n, el, threads, sample = oracle_sample(w, 0, steps=args.steps, warmup=args.warmup)
+    line = {"metric": METRIC, "value": rate, "unit": UNIT, "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * el / n, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "layers": w.layers, "batch": w.B,
+                       "ctx": w.seq_lens[0], "step": "one sequence, layer 0 (bounded sample)"},
+            "cpu_baseline": {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU stack
+class Stack:
+    """All layers of a workload on one GPU, with per-step inputs resident."""
+
+    def __init__(self, w: wl.Workload, dev, total_steps: int, seed_offset: int):
+        from long_context_decoding_b200 import csa
+        self.csa = csa
+        self.w = w = replace(w, steps=total_steps, seed=w.seed + seed_offset)
+        self.dev = dev
+        self.d = csa.make_dims(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.num_pages, w.max_sel)
+        self.ws = csa.new_workspace(self.d, dev)
+        self.layers = []
+        for i in range(w.layers):
+            c = wl.make_case(w, dev, layer=i)
+            lay = csa.Layer(self.d, c.k_cache, c.v_cache, c.page_table, c.seq_lens, w.prefix,
+                            c.window, c.budget, ws=self.ws)
+            lay.rebuild_meta()
+            lay.case = c
+            self.layers.append(lay)
+        L0 = torch.tensor(w.seq_lens, dtype=torch.int32, device=dev)
+        self.lens = [(L0 + s + 1).contiguous() for s in range(total_steps)]
+        self.inputs = [[wl.step_tokens(lay.case, s) for lay in self.layers]
+                       for s in range(total_steps)]
+        torch.cuda.synchronize()
+        assert csa.device_status(self.ws) == 0
+
+    def calls(self, s: int, q=None, nk=None, nv=None, what="all", layers=None):
+        csa = self.csa
+        for li in (layers if layers is not None else range(len(self.layers))):
+            lay = self.layers[li]
+            q_, nk_, nv_ = self.inputs[s][li]
+            q_ = q[li] if q is not None else q_
+            nk_ = nk[li] if nk is not None else nk_
+            nv_ = nv[li] if nv is not None else nv_
+            lens = self.lens[s]
+            if what in ("all",):
+                csa.meta_update(self.d, lay.k_cache, lay.v_cache, lay.meta, lay.page_table, lens,
+                                nk_, nv_, 1, self.ws)
+            if what in ("all", "select"):
+                csa.score_select(self.d, q_, lay.meta, lay.page_table, lens, lay.prefix,
+                                 lay.window, lay.budget, lay.sel, lay.n_sel, self.ws)
+            if what in ("all", "decode"):
+                csa.decode(self.d, q_, lay.k_cache, lay.v_cache, lay.page_table, lens, lay.sel,
+                           lay.n_sel, lay.prefix, lay.window, lay.out, self.ws, lay.lse)
+
+    def launches_per_step(self) -> int:
+        n = 0
+        for lay in self.layers:
+            n += 1 + 1 + (1 if lay.budget // 16 > 0 else 0) + 1
+        return n
+
+    def graph(self, fn):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                fn()
+        torch.cuda.current_stream().wait_stream(s)
+        return g
+
+    def bytes_per_layer(self, s: int):
+        """Algorithmic bytes of each layer at step s."""
+        L = [x + s + 1 for x in self.w.seq_lens]
+        return [cost.layer_bytes(L, self.w.Hq, self.w.Hkv, self.w.D, lay.prefix, lay.window,
+                                 lay.budget) for lay in self.layers]
+
+
+def time_graphs(graphs, reps=1):
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        for g in graphs:
+            g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / 1000.0
+
+
+def run_ours(args, dist: Dist, base: wl.Workload):
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the CUDA path has no CPU fallback)")
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    K, W = args.steps, args.warmup
+    st = Stack(base, dev, K + W, seed_offset=1000 * dist.rank)
+    w = st.w
+    nl = len(st.layers)
+    # eager pass over every step: sets kernel attributes, checks the flags
+    for s in range(K + W):
+        st.calls(s)
+    torch.cuda.synchronize()
+    assert st.csa.device_status(st.ws) == 0, "device flag after the eager pass"
+    graphs = [st.graph(lambda s=s: st.calls(s)) for s in range(K + W)]
+    for s in range(W):
+        graphs[s].replay()
+    clocks = None if args.profile else Clocks(dev)
+    if clocks:   # ~1 s of untimed load so that the sampler sees the clock under load
+        t_end = time.perf_counter() + 1.0
+        while time.perf_counter() < t_end:
+            for g in graphs[:W]:
+                g.replay()
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    dist.barrier()
+    t = time_graphs(graphs[W:W + K])
+    dist.barrier()
+    clk = clocks.stop() if clocks else None
+    t = dist.max(t)
+    flags = st.csa.device_status(st.ws)
+    value = dist.world * w.B * nl * K / t
+    t_layer = t / (K * nl)
+
+    # per-layer algorithmic bytes over the timed steps (averaged)
+    per_layer = [st.bytes_per_layer(s) for s in range(W, W + K)]
+    layer_sparse = statistics.mean(sum(x["sparse"] for x in bl) / nl for bl in per_layer)
+    meta_b = statistics.mean(sum(x["meta"] for x in bl) / nl for bl in per_layer)
+    kv_b = statistics.mean(sum(x["kv"] + x["q_out"] for x in bl) / nl for bl in per_layer)
+    peak, peak_kind = hbm_peak()
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": K,
+            "warmup": W, "ms_per_step": 1000 * t / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian q/K/V, random page permutation)",
+            "config": {"workload": w.name, "layers": nl, "batch": w.B, "ctx": w.seq_lens[0],
+                       "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,
+                       "prefix": w.prefix,
+                       "window_budget": [[lay.window, lay.budget] for lay in st.layers],
+                       "l2": "no flush: every layer moves > 126 MB (L2); "
+                             f"{layer_sparse * nl / 1e9:.2f} GB per step",
+                       "timing": "one CUDA graph per decode step, K graphs replayed between "
+                                 "CUDA events; max over ranks"},
+            "gpu_launches": st.launches_per_step() * K,
+            "layer_step": {"us": 1e6 * t_layer, "algorithmic_bytes": layer_sparse,
+                           "achieved_gbs": layer_sparse / t_layer / 1e9,
+                           "frac_of_measured_peak": layer_sparse / t_layer / 1e9 / peak,
+                           "frac_of_8tbs_nominal": layer_sparse / t_layer / 1e9 / NOMINAL_HBM_GBS},
+            "device_flags": flags}
+
+    if not args.profile:
+        # ---- per-call timing: graph replays over all layers (inputs >> L2)
+        s_last = W + K - 1
+        g_sel = st.graph(lambda: st.calls(s_last, what="select"))
+        g_dec = st.graph(lambda: st.calls(s_last, what="decode"))
+        reps = 5
+        time_graphs([g_sel])
+        t_sel = time_graphs([g_sel], reps) / (reps * nl)
+        time_graphs([g_dec])
+        t_dec = time_graphs([g_dec], reps) / (reps * nl)
+        bl = st.bytes_per_layer(s_last)
+        sel_bytes = sum(x["meta"] for x in bl) / nl
+        dec_bytes = sum(x["kv"] + x["q_out"] for x in bl) / nl
+        calls = {"score_select": {"us": 1e6 * t_sel, "bytes": sel_bytes,
+                                  "gbs": sel_bytes / t_sel / 1e9},
+                 "decode": {"us": 1e6 * t_dec, "bytes": dec_bytes,
+                            "gbs": dec_bytes / t_dec / 1e9}}
+        dom = max(calls, key=lambda k: calls[k]["us"])
+        ach = calls[dom]["gbs"]
+        line["roofline"] = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak,
+                            "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
+                            "traffic": None,
+                            "note": "achieved = algorithmic bytes of the call (metadata of the "
+                                    "candidate pages for score_select; K/V of the attended "
+                                    "tokens + q/out for decode) / CUDA-event time per call, "
+                                    "graph replay over the 12 layers; score_select covers the "
+                                    "scoring and the top-k kernels"}
+        line["calls"] = calls
+        line["clocks"] = clk
+
+        # ---- end to end through the C ABI from pinned host buffers
+        if not args.no_e2e:
+            line["e2e"] = e2e(st, K, W, dist)
+
+        # ---- 64k single layer (the other context of the metric)
+        if not args.no_secondary and base.name == wl.CTX256K.name:
+            line["ctx64k"] = secondary_64k(dev, dist)
+
+        # ---- CPU oracle on a bounded sample
+        if not args.no_cpu_baseline and dist.rank == 0 and dist.world == 1:
+            rate, n, el, threads, sample = oracle_sample(base, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads,
+                                    "kind": "oracle", "sample": sample}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def e2e(st: Stack, K: int, W: int, dist: Dist):
+    """Per step: H2D copy of the step's q/new_k/new_v (pinned host memory),
+    the 36 library calls, D2H copy of every layer's output; one CUDA graph
+    per step, K steps timed."""
+    nl = len(st.layers)
+    host_in, dev_in, host_out = [], [], []
+    for s in range(K + W):
+        hi = [[t.cpu().pin_memory() for t in st.inputs[s][li]] for li in range(nl)]
+        di = [[torch.empty_like(t) for t in st.inputs[s][li]] for li in range(nl)]
+        ho = [torch.empty(st.layers[li].out.shape, dtype=torch.bfloat16).pin_memory()
+              for li in range(nl)]
+        host_in.append(hi), dev_in.append(di), host_out.append(ho)
+
+    def step(s):
+        for li in range(nl):
+            for d_, h_ in zip(dev_in[s][li], host_in[s][li]):
+                d_.copy_(h_, non_blocking=True)
+        st.calls(s, q=[x[0] for x in dev_in[s]], nk=[x[1] for x in dev_in[s]],
+                 nv=[x[2] for x in dev_in[s]])
+        for li in range(nl):
+            host_out[s][li].copy_(st.layers[li].out, non_blocking=True)
+
+    graphs = [st.graph(lambda s=s: step(s)) for s in range(K + W)]
+    for s in range(W):
+        graphs[s].replay()
+    torch.cuda.synchronize()
+    dist.barrier()
+    t = dist.max(time_graphs(graphs[W:W + K]))
+    h2d = sum(t_.numel() * t_.element_size() for li in range(nl) for t_ in host_in[0][li])
+    d2h = sum(t_.numel() * t_.element_size() for t_ in host_out[0])
+    return {"value": dist.world * st.w.B * nl * K / t, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "path": "pinned host -> device copies, csa_meta_update / csa_score_select / "
+                    "csa_decode per layer, device -> pinned host copy of out; one CUDA graph "
+                    "per step"}
+
+
+def secondary_64k(dev, dist: Dist):
+    """The 64k single-layer workload: one layer step (score + select +
+    decode, no append) per graph; a 256 MB scrub write between replays
+    flushes L2 (the layer itself moves only ~84 MB)."""
+    from long_context_decoding_b200 import csa
+    w = wl.CTX64K
+    c = wl.make_case(w, dev)
+    d = csa.make_dims(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.num_pages, w.max_sel)
+    lay = csa.Layer(d, c.k_cache, c.v_cache, c.page_table, c.seq_lens, w.prefix, w.window,
+                    w.budget)
+    lay.rebuild_meta()
+    scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def body():
+        lay.step(c.q)
+
+    body()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            body()
+    torch.cuda.current_stream().wait_stream(s)
+    times = []
+    for i in range(30):
+        scrub.fill_(i & 0xff)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 5:
+            times.append(a.elapsed_time(b) / 1000.0)
+    t = dist.max(statistics.median(times))
+    by = cost.layer_bytes(w.seq_lens, w.Hq, w.Hkv, w.D, w.prefix, w.window, w.budget)
+    peak, _ = hbm_peak()
+    ach = by["sparse"] / t / 1e9
+    # dense comparison on the same cache
+    out = torch.empty_like(lay.out)
+
+    def dense():
+        csa.decode_full(d, c.q, c.k_cache, c.v_cache, c.page_table, c.seq_lens, out, lay.ws)
+
+    dense()
+    torch.cuda.synchronize()
+    dt = []
+    for i in range(15):
+        scrub.fill_(i & 0xff)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dense()
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            dt.append(a.elapsed_time(b) / 1000.0)
+    tdn = statistics.median(dt)
+    return {"workload": w.name, "value": dist.world * w.B / t, "unit": UNIT,
+            "us_per_layer_step": 1e6 * t, "algorithmic_bytes": by["sparse"],
+            "achieved_gbs": ach, "frac_of_measured_peak": ach / peak,
+            "frac_of_8tbs_nominal": ach / NOMINAL_HBM_GBS,
+            "dense_us": 1e6 * tdn, "dense_gbs": by["dense"] / tdn / 1e9,
+            "speedup_vs_dense": tdn / t,
+            "timing": "median of 25 graph replays, 256 MB L2 scrub between replays"}
+
+
+def main():
+    args = parse_args()
+    dist = Dist()
+    base = wl.CTX256K if args.workload == "ctx256k" else replace(wl.CTX64K, steps=0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, dist, base)
+        else:
+            run_ours(args, dist, base)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

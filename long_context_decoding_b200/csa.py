@@ -1,0 +1,218 @@
+"""Python binding of libcsa.so (C ABI in include/csa.h).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels of libcsa.so.  Tensors are torch CUDA tensors; the calls run on the
+current torch stream (or the one passed).  There is no CPU fallback: if the
+library is missing or no CUDA device is present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+PAGE = 16
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_OK = 0
+CSA_ERR_DEVICE_FLAG = -5
+DEVFLAG_BAD_PAGE_ID = 1
+DEVFLAG_BAD_SELECTION = 2
+DEVFLAG_BAD_SEQ_LEN = 4
+DEVFLAG_TIMEOUT = 8
+
+EXPORTS = ("csa_version", "csa_status_string", "csa_workspace_size", "csa_workspace_init",
+           "csa_meta_update", "csa_score_select", "csa_decode", "csa_decode_full",
+           "csa_get_device_status")
+
+
+class CsaError(RuntimeError):
+    def __init__(self, where: str, status: int, msg: str):
+        super().__init__(f"{where}: {msg} (status {status})")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    """Mirror of ``csa_dims``."""
+
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("D", ctypes.c_int), ("page_size", ctypes.c_int),
+                ("max_pages_per_seq", ctypes.c_int), ("num_pages", ctypes.c_int),
+                ("max_sel", ctypes.c_int)]
+
+    def __repr__(self):
+        return "Dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def make_dims(B, Hq, Hkv, D, max_pages_per_seq, num_pages, max_sel, page_size=PAGE) -> Dims:
+    return Dims(B, Hq, Hkv, D, page_size, max_pages_per_seq, num_pages, max_sel)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcsa.so (raises when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m long_context_decoding_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        D = ctypes.POINTER(Dims)
+        L.csa_version.restype = I
+        L.csa_status_string.argtypes = [I]
+        L.csa_status_string.restype = ctypes.c_char_p
+        L.csa_workspace_size.argtypes = [D]
+        L.csa_workspace_size.restype = Z
+        L.csa_workspace_init.argtypes = [P, Z, P]
+        L.csa_meta_update.argtypes = [D, P, P, P, P, P, P, P, I, P, Z, P]
+        L.csa_score_select.argtypes = [D, P, P, P, P, I, I, I, P, P, P, P, Z, P]
+        L.csa_decode.argtypes = [D, P, P, P, P, P, P, P, I, I, ctypes.c_float, P, P, P, Z, P]
+        L.csa_decode_full.argtypes = [D, P, P, P, P, P, ctypes.c_float, P, P, P, Z, P]
+        L.csa_get_device_status.argtypes = [P, P, ctypes.POINTER(I)]
+        for f in ("csa_workspace_init", "csa_meta_update", "csa_score_select", "csa_decode",
+                  "csa_decode_full", "csa_get_device_status"):
+            getattr(L, f).restype = I
+        _lib = L
+    return _lib
+
+
+def status_string(st: int) -> str:
+    return lib().csa_status_string(int(st)).decode()
+
+
+def _check(where: str, st: int):
+    if st != CSA_OK:
+        raise CsaError(where, st, status_string(st))
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(d: Dims) -> int:
+    n = lib().csa_workspace_size(ctypes.byref(d))
+    if n == 0:
+        raise CsaError("csa_workspace_size", -2, "invalid or unsupported shape")
+    return int(n)
+
+
+def new_workspace(d: Dims, device="cuda", stream=None) -> torch.Tensor:
+    """Allocate (with torch) and zero a workspace for shape ``d``."""
+    ws = torch.empty(workspace_size(d), dtype=torch.uint8, device=device)
+    _check("csa_workspace_init",
+           lib().csa_workspace_init(_ptr(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def meta_update(d: Dims, k_cache, v_cache, meta, page_table, seq_lens, new_k, new_v, n_new: int,
+                ws, stream=None):
+    """Append n_new tokens per sequence (new_k/new_v None: rebuild metadata)."""
+    bf = torch.bfloat16
+    _check("csa_meta_update", lib().csa_meta_update(
+        ctypes.byref(d), _ptr(k_cache, bf, "k_cache"), _ptr(v_cache, bf, "v_cache"),
+        _ptr(meta, bf, "meta"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(new_k, bf, "new_k"),
+        _ptr(new_v, bf, "new_v"), int(n_new), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def score_select(d: Dims, q, meta, page_table, seq_lens, prefix: int, window: int, budget: int,
+                 sel, n_sel, ws, scores_out=None, stream=None):
+    """Quest scores from metadata and top-k page selection into sel / n_sel."""
+    bf = torch.bfloat16
+    _check("csa_score_select", lib().csa_score_select(
+        ctypes.byref(d), _ptr(q, bf, "q"), _ptr(meta, bf, "meta"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        int(prefix), int(window), int(budget), _ptr(sel, torch.int32, "sel"),
+        _ptr(n_sel, torch.int32, "n_sel"), _ptr(scores_out, torch.float32, "scores_out"),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def decode(d: Dims, q, k_cache, v_cache, page_table, seq_lens, sel, n_sel, prefix: int,
+           window: int, out, ws, lse=None, scale: float = 0.0, stream=None):
+    """Combined sparse attention over prefix + window + selected pages."""
+    bf = torch.bfloat16
+    _check("csa_decode", lib().csa_decode(
+        ctypes.byref(d), _ptr(q, bf, "q"), _ptr(k_cache, bf, "k_cache"),
+        _ptr(v_cache, bf, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(sel, torch.int32, "sel"),
+        _ptr(n_sel, torch.int32, "n_sel"), int(prefix), int(window), float(scale),
+        _ptr(out, bf, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def decode_full(d: Dims, q, k_cache, v_cache, page_table, seq_lens, out, ws, lse=None,
+                scale: float = 0.0, stream=None):
+    """Dense decode over every valid token (the unmodified layer)."""
+    bf = torch.bfloat16
+    _check("csa_decode_full", lib().csa_decode_full(
+        ctypes.byref(d), _ptr(q, bf, "q"), _ptr(k_cache, bf, "k_cache"),
+        _ptr(v_cache, bf, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), float(scale), _ptr(out, bf, "out"),
+        _ptr(lse, torch.float32, "lse"), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def device_status(ws, stream=None) -> int:
+    """Synchronise, return and clear the device flag bits (0 = clean)."""
+    flags = ctypes.c_int(0)
+    st = lib().csa_get_device_status(_ptr(ws), _stream(stream), ctypes.byref(flags))
+    if st not in (CSA_OK, CSA_ERR_DEVICE_FLAG):
+        _check("csa_get_device_status", st)
+    return int(flags.value)
+
+
+class Layer:
+    """Device state of one full-attention layer: a paged cache, its page
+    metadata, the page table, sequence lengths and the per-layer
+    (prefix, window, budget).  ``step`` runs one decode step through the
+    C ABI: append + metadata update, score + select, sparse decode."""
+
+    def __init__(self, d: Dims, k_cache, v_cache, page_table, seq_lens, prefix: int, window: int,
+                 budget: int, meta=None, ws=None):
+        self.d = d
+        dev = k_cache.device
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.page_table, self.seq_lens = page_table, seq_lens
+        self.prefix, self.window, self.budget = prefix, window, budget
+        self.meta = meta if meta is not None else torch.zeros(
+            (d.num_pages, d.Hkv, 2, d.D), dtype=torch.bfloat16, device=dev)
+        self.ws = ws if ws is not None else new_workspace(d, dev)
+        self.sel = torch.zeros((d.B, d.Hkv, d.max_sel), dtype=torch.int32, device=dev)
+        self.n_sel = torch.zeros((d.B, d.Hkv), dtype=torch.int32, device=dev)
+        self.out = torch.empty((d.B, d.Hq, d.D), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((d.B, d.Hq), dtype=torch.float32, device=dev)
+
+    def rebuild_meta(self, stream=None):
+        n = self.d.max_pages_per_seq * PAGE
+        meta_update(self.d, self.k_cache, self.v_cache, self.meta, self.page_table, self.seq_lens,
+                    None, None, n, self.ws, stream)
+
+    def step(self, q, new_k=None, new_v=None, stream=None):
+        """One decode step.  With new_k/new_v ([B][1][Hkv][D]) the token is
+        appended first; seq_lens must already count it."""
+        if new_k is not None:
+            meta_update(self.d, self.k_cache, self.v_cache, self.meta, self.page_table,
+                        self.seq_lens, new_k, new_v, new_k.shape[1], self.ws, stream)
+        score_select(self.d, q, self.meta, self.page_table, self.seq_lens, self.prefix,
+                     self.window, self.budget, self.sel, self.n_sel, self.ws, stream=stream)
+        decode(self.d, q, self.k_cache, self.v_cache, self.page_table, self.seq_lens, self.sel,
+               self.n_sel, self.prefix, self.window, self.out, self.ws, self.lse, stream=stream)
+        return self.out

@@ -1,0 +1,340 @@
+// csa_api.cu -- the C ABI of libcsa.so (declared in include/csa.h).
+//
+// Host-side only: argument validation, the workspace layout, TMA tensor-map
+// encoding and kernel dispatch.  No memory is allocated here; every buffer
+// belongs to the caller.
+#include <math.h>
+#include <mutex>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace csa {
+
+int device_sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 148;
+    }
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WsLayout workspace_layout(const Shape& s) {
+    WsLayout w;
+    const size_t units = (size_t)s.B * s.Hkv;
+    size_t off = 0;
+    w.flags = off;
+    off = align_up(off + 4, 256);
+    w.score_tickets = off;
+    off = align_up(off + 4 * units, 256);
+    w.dec_tickets = off;
+    off = align_up(off + 4 * units, 256);
+    w.scores = off;
+    off = align_up(off + 4 * units * (size_t)s.MP, 256);
+    w.partials = off;
+    w.dec_slots = (size_t)decode_grid(s) + units;
+    off = align_up(off + 4 * w.dec_slots * (size_t)s.G * (s.D + 2), 256);
+    w.total = off;
+    return w;
+}
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// A [num_pages * Hkv * 16][D] bf16 view of a paged cache; boxes of
+// 64 channels x 16 tokens (one page of one kv-head, half or quarter of D),
+// 128-byte swizzle.
+static bool make_cache_map(CUtensorMap* m, const void* base, const Shape& s) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)s.D, (cuuint64_t)s.NPG * s.Hkv * kPage};
+    cuuint64_t strides[1] = {(cuuint64_t)s.D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kPage};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- validation
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static int check_dims(const csa_dims* d, Shape* s) {
+    if (!d) return CSA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->D < 1 || d->max_pages_per_seq < 1 ||
+        d->num_pages < 1 || d->max_sel < 1)
+        return CSA_ERR_INVALID_ARG;
+    if (d->Hq % d->Hkv != 0) return CSA_ERR_INVALID_ARG;
+    if (d->page_size != kPage) return CSA_ERR_UNSUPPORTED;
+    if (d->D != 64 && d->D != 128 && d->D != 256) return CSA_ERR_UNSUPPORTED;
+    const int G = d->Hq / d->Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return CSA_ERR_UNSUPPORTED;
+    if ((long long)d->B * d->Hkv > kMaxUnits) return CSA_ERR_UNSUPPORTED;
+    if ((long long)d->num_pages * d->Hkv * kPage >= (1ll << 31)) return CSA_ERR_UNSUPPORTED;
+    if ((long long)d->max_pages_per_seq * kPage >= (1ll << 31)) return CSA_ERR_UNSUPPORTED;
+    s->B = d->B;
+    s->Hq = d->Hq;
+    s->Hkv = d->Hkv;
+    s->G = G;
+    s->D = d->D;
+    s->MP = d->max_pages_per_seq;
+    s->NPG = d->num_pages;
+    s->max_sel = d->max_sel;
+    return CSA_OK;
+}
+
+#define CSA_REQUIRE(ptr)                                  \
+    do {                                                  \
+        if (!(ptr) || !aligned16(ptr)) return CSA_ERR_INVALID_ARG; \
+    } while (0)
+#define CSA_OPTIONAL(ptr)                                 \
+    do {                                                  \
+        if ((ptr) && !aligned16(ptr)) return CSA_ERR_INVALID_ARG; \
+    } while (0)
+
+static int check_ws(const Shape& s, void* ws, size_t bytes, WsLayout* w) {
+    if (!ws || !aligned16(ws)) return CSA_ERR_WORKSPACE;
+    *w = workspace_layout(s);
+    if (bytes < w->total) return CSA_ERR_WORKSPACE;
+    return CSA_OK;
+}
+
+static int launch_status(cudaError_t e) {
+    if (e == cudaSuccess) return CSA_OK;
+    cudaGetLastError();
+    return CSA_ERR_CUDA;
+}
+
+template <typename T>
+static T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+int csa_version(void) { return 100; }
+
+const char* csa_status_string(int st) {
+    switch (st) {
+        case CSA_OK: return "ok";
+        case CSA_ERR_INVALID_ARG: return "invalid argument";
+        case CSA_ERR_UNSUPPORTED: return "unsupported shape";
+        case CSA_ERR_WORKSPACE: return "workspace missing or too small";
+        case CSA_ERR_CUDA: return "CUDA error";
+        case CSA_ERR_DEVICE_FLAG: return "device-side error flag set";
+        default: return "unknown status";
+    }
+}
+
+size_t csa_workspace_size(const csa_dims* d) {
+    Shape s;
+    if (check_dims(d, &s) != CSA_OK) return 0;
+    return workspace_layout(s).total;
+}
+
+int csa_workspace_init(void* workspace, size_t bytes, void* stream) {
+    if (!workspace || !aligned16(workspace)) return CSA_ERR_WORKSPACE;
+    return launch_status(cudaMemsetAsync(workspace, 0, bytes, (cudaStream_t)stream));
+}
+
+int csa_meta_update(const csa_dims* d, void* k_cache, void* v_cache, void* meta,
+                    const int32_t* page_table, const int32_t* seq_lens, const void* new_k,
+                    const void* new_v, int n_new, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+    Shape s;
+    int rc = check_dims(d, &s);
+    if (rc != CSA_OK) return rc;
+    CSA_REQUIRE(meta);
+    CSA_REQUIRE(page_table);
+    CSA_REQUIRE(seq_lens);
+    CSA_REQUIRE(k_cache);
+    if (n_new < 1) return CSA_ERR_INVALID_ARG;
+    if ((new_k == nullptr) != (new_v == nullptr)) return CSA_ERR_INVALID_ARG;
+    if (new_k) {
+        CSA_REQUIRE(v_cache);
+        CSA_REQUIRE(new_k);
+        CSA_REQUIRE(new_v);
+        if ((long long)n_new > (long long)s.MP * kPage) return CSA_ERR_INVALID_ARG;
+    }
+    WsLayout w;
+    rc = check_ws(s, workspace, workspace_bytes, &w);
+    if (rc != CSA_OK) return rc;
+    MetaParams p;
+    p.k_cache = static_cast<uint16_t*>(k_cache);
+    p.v_cache = static_cast<uint16_t*>(v_cache);
+    p.meta = static_cast<uint16_t*>(meta);
+    p.page_table = page_table;
+    p.seq_lens = seq_lens;
+    p.new_k = static_cast<const uint16_t*>(new_k);
+    p.new_v = static_cast<const uint16_t*>(new_v);
+    p.n_new = n_new;
+    p.flags = at<uint32_t>(workspace, w.flags);
+    p.s = s;
+    return launch_status(launch_meta_update(p, (cudaStream_t)stream));
+}
+
+int csa_score_select(const csa_dims* d, const void* q, const void* meta,
+                     const int32_t* page_table, const int32_t* seq_lens, int prefix, int window,
+                     int budget_tokens, int32_t* sel_pages, int32_t* n_sel, float* scores_out,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+    Shape s;
+    int rc = check_dims(d, &s);
+    if (rc != CSA_OK) return rc;
+    CSA_REQUIRE(q);
+    CSA_REQUIRE(meta);
+    CSA_REQUIRE(page_table);
+    CSA_REQUIRE(seq_lens);
+    CSA_REQUIRE(sel_pages);
+    CSA_REQUIRE(n_sel);
+    CSA_OPTIONAL(scores_out);
+    if (prefix < 0 || window < 0 || budget_tokens < 0) return CSA_ERR_INVALID_ARG;
+    const int k_pages = budget_tokens / kPage;
+    if (k_pages > s.max_sel) return CSA_ERR_INVALID_ARG;
+    WsLayout w;
+    rc = check_ws(s, workspace, workspace_bytes, &w);
+    if (rc != CSA_OK) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    ScoreParams sp;
+    sp.q = static_cast<const uint16_t*>(q);
+    sp.meta = static_cast<const uint16_t*>(meta);
+    sp.page_table = page_table;
+    sp.seq_lens = seq_lens;
+    sp.prefix = prefix;
+    sp.window = window;
+    sp.scores_ws = at<float>(workspace, w.scores);
+    sp.scores_out = scores_out;
+    sp.flags = at<uint32_t>(workspace, w.flags);
+    sp.s = s;
+    if (k_pages > 0 || scores_out) {
+        rc = launch_status(launch_score(sp, st));
+        if (rc != CSA_OK) return rc;
+    }
+    SelectParams lp;
+    lp.scores_ws = sp.scores_ws;
+    lp.seq_lens = seq_lens;
+    lp.prefix = prefix;
+    lp.window = window;
+    lp.k_pages = k_pages;
+    lp.sel = sel_pages;
+    lp.n_sel = n_sel;
+    lp.flags = sp.flags;
+    lp.smem_keys = 0;
+    lp.s = s;
+    return launch_status(launch_select(lp, st));
+}
+
+static int decode_common(const csa_dims* d, const void* q, const void* k_cache,
+                         const void* v_cache, const int32_t* page_table, const int32_t* seq_lens,
+                         const int32_t* sel_pages, const int32_t* n_sel, int prefix, int window,
+                         int dense, float scale, void* out, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    Shape s;
+    int rc = check_dims(d, &s);
+    if (rc != CSA_OK) return rc;
+    CSA_REQUIRE(q);
+    CSA_REQUIRE(k_cache);
+    CSA_REQUIRE(v_cache);
+    CSA_REQUIRE(page_table);
+    CSA_REQUIRE(seq_lens);
+    CSA_REQUIRE(out);
+    CSA_OPTIONAL(lse);
+    if (!dense) {
+        CSA_REQUIRE(sel_pages);
+        CSA_REQUIRE(n_sel);
+        if (prefix < 0 || window < 0) return CSA_ERR_INVALID_ARG;
+    }
+    if (!(scale == scale) || isinf(scale)) return CSA_ERR_INVALID_ARG;
+    WsLayout w;
+    rc = check_ws(s, workspace, workspace_bytes, &w);
+    if (rc != CSA_OK) return rc;
+    CUtensorMap tmK, tmV;
+    if (!make_cache_map(&tmK, k_cache, s) || !make_cache_map(&tmV, v_cache, s))
+        return CSA_ERR_CUDA;
+    DecodeParams p;
+    p.q = static_cast<const uint16_t*>(q);
+    p.page_table = page_table;
+    p.seq_lens = seq_lens;
+    p.sel = sel_pages;
+    p.n_sel = n_sel;
+    p.prefix = prefix;
+    p.window = window;
+    p.dense = dense;
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)s.D);
+    p.scale_log2 = sc * 1.4426950408889634f;
+    p.out = static_cast<uint16_t*>(out);
+    p.lse = lse;
+    p.flags = at<uint32_t>(workspace, w.flags);
+    p.tickets = at<uint32_t>(workspace, w.dec_tickets);
+    p.partials = at<float>(workspace, w.partials);
+    p.s = s;
+    return launch_status(launch_decode(p, tmK, tmV, (cudaStream_t)stream));
+}
+
+int csa_decode(const csa_dims* d, const void* q, const void* k_cache, const void* v_cache,
+               const int32_t* page_table, const int32_t* seq_lens, const int32_t* sel_pages,
+               const int32_t* n_sel, int prefix, int window, float scale, void* out, float* lse,
+               void* workspace, size_t workspace_bytes, void* stream) {
+    return decode_common(d, q, k_cache, v_cache, page_table, seq_lens, sel_pages, n_sel, prefix,
+                         window, 0, scale, out, lse, workspace, workspace_bytes, stream);
+}
+
+int csa_decode_full(const csa_dims* d, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* page_table, const int32_t* seq_lens, float scale, void* out,
+                    float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    return decode_common(d, q, k_cache, v_cache, page_table, seq_lens, nullptr, nullptr, 0, 0, 1,
+                         scale, out, lse, workspace, workspace_bytes, stream);
+}
+
+int csa_get_device_status(void* workspace, void* stream, int* flags_out) {
+    if (!workspace || !aligned16(workspace)) return CSA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t flags = 0;
+    if (cudaMemcpyAsync(&flags, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    if (flags_out) *flags_out = (int)flags;
+    return flags ? CSA_ERR_DEVICE_FLAG : CSA_OK;
+}
+
+}  // extern "C"

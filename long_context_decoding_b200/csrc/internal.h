@@ -1,0 +1,94 @@
+// internal.h -- host-side interface between the C ABI (csa_api.cu) and the
+// kernel translation units.  Not installed; the public ABI is include/csa.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace csa {
+
+// Workspace layout (byte offsets into the caller's workspace).
+struct WsLayout {
+    size_t flags;          // uint32 device flag word
+    size_t score_tickets;  // uint32 [units]
+    size_t dec_tickets;    // uint32 [units]
+    size_t scores;         // fp32 [B][Hkv][max_pages]
+    size_t partials;       // fp32 [dec_slots][G][D + 2]
+    size_t dec_slots;      // partial records available
+    size_t total;
+};
+
+struct Shape {
+    int B, Hq, Hkv, G, D, MP, NPG, max_sel;
+};
+
+// ---------------------------------------------------------------- meta
+struct MetaParams {
+    uint16_t* k_cache;
+    uint16_t* v_cache;
+    uint16_t* meta;
+    const int32_t* page_table;
+    const int32_t* seq_lens;
+    const uint16_t* new_k;   // nullable (rebuild)
+    const uint16_t* new_v;
+    int n_new;
+    uint32_t* flags;
+    Shape s;
+};
+cudaError_t launch_meta_update(const MetaParams& p, cudaStream_t st);
+
+// ---------------------------------------------------------------- score
+struct ScoreParams {
+    const uint16_t* q;
+    const uint16_t* meta;
+    const int32_t* page_table;
+    const int32_t* seq_lens;
+    int prefix, window;
+    float* scores_ws;       // [B][Hkv][MP]
+    float* scores_out;      // nullable
+    uint32_t* flags;
+    Shape s;
+};
+cudaError_t launch_score(const ScoreParams& p, cudaStream_t st);
+
+// ---------------------------------------------------------------- select
+struct SelectParams {
+    float* scores_ws;       // read; rewritten in place as order keys
+    const int32_t* seq_lens;
+    int prefix, window, k_pages;
+    int32_t* sel;
+    int32_t* n_sel;
+    uint32_t* flags;
+    int smem_keys;          // set by the launcher
+    Shape s;
+};
+cudaError_t launch_select(const SelectParams& p, cudaStream_t st);
+
+// ---------------------------------------------------------------- decode
+struct DecodeParams {
+    const uint16_t* q;
+    const int32_t* page_table;
+    const int32_t* seq_lens;
+    const int32_t* sel;     // nullable when dense
+    const int32_t* n_sel;
+    int prefix, window;
+    int dense;
+    float scale_log2;       // softmax scale * log2(e)
+    uint16_t* out;
+    float* lse;             // nullable
+    uint32_t* flags;
+    uint32_t* tickets;      // [units]
+    float* partials;        // [dec_slots][G][D + 2]
+    Shape s;
+};
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                          cudaStream_t st);
+
+// Grid sizes (shared by the workspace sizing and the launches).
+int device_sm_count();
+int decode_grid(const Shape& s);
+WsLayout workspace_layout(const Shape& s);
+
+}  // namespace csa

@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every symbol include/csa.h declares, and
+rejects bad arguments on the host (no GPU needed: every case below returns
+before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_decoding_b200 import build as csa_build
+from long_context_decoding_b200 import csa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    csa_build.build()
+    return csa.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "csa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(csa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert header_functions() == sorted(csa.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in header_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_version(L):
+    assert L.csa_version() == 100
+    assert csa.status_string(0) == "ok"
+    assert "workspace" in csa.status_string(-3)
+    assert csa.status_string(-99) == "unknown status"
+
+
+def dims(**kw):
+    base = dict(B=4, Hq=32, Hkv=4, D=128, max_pages_per_seq=16388, num_pages=65555, max_sel=512)
+    base.update(kw)
+    return csa.make_dims(**base)
+
+
+def test_workspace_size_valid_and_invalid(L):
+    n = csa.workspace_size(dims())
+    # scores alone need B*Hkv*max_pages*4 bytes
+    assert n >= 4 * 4 * 16388 * 4
+    for bad in (dict(D=96), dict(Hq=12, Hkv=4), dict(Hq=30, Hkv=4), dict(B=0),
+                dict(B=1024, Hkv=4, Hq=4)):
+        with pytest.raises(csa.CsaError):
+            csa.workspace_size(dims(**bad))
+    d = dims()
+    d.page_size = 32
+    assert L.csa_workspace_size(ctypes.byref(d)) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)        # 16-byte aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def test_host_validation_codes(L):
+    d = dims()
+    P = [FAKE] * 6
+    W = (FAKE, ctypes.c_size_t(1 << 40), None)          # workspace, bytes, stream
+
+    def score(q=FAKE, budget=64, ws=W):
+        return L.csa_score_select(ctypes.byref(d), q, FAKE, FAKE, FAKE, 0, 0, budget, FAKE, FAKE,
+                                  None, *ws)
+    assert score(q=None) == -1                      # null pointer
+    assert score(q=MISALIGNED) == -1                # not 16-byte aligned
+    assert score(budget=-16) == -1                  # negative budget
+    assert score(budget=16 * 513) == -1             # more pages than max_sel
+    assert score(ws=(None, ctypes.c_size_t(1 << 40), None)) == -3
+    assert score(ws=(FAKE, ctypes.c_size_t(16), None)) == -3
+    # unsupported head dim / group size
+    bad = dims(D=80)
+    assert L.csa_decode_full(ctypes.byref(bad), *P[:5], ctypes.c_float(0), FAKE, None, FAKE,
+                             1 << 40, None) == -2
+    bad = dims(Hq=12, Hkv=4)
+    assert L.csa_decode(ctypes.byref(bad), *P[:5], FAKE, FAKE, 0, 0, ctypes.c_float(0), FAKE,
+                        None, FAKE, 1 << 40, None) == -2
+    # sparse decode needs a selection; NaN scale is rejected
+    assert L.csa_decode(ctypes.byref(d), *P[:5], None, FAKE, 0, 0, ctypes.c_float(0), FAKE, None,
+                        FAKE, 1 << 40, None) == -1
+    assert L.csa_decode_full(ctypes.byref(d), *P[:5], ctypes.c_float(float("nan")), FAKE, None,
+                             FAKE, 1 << 40, None) == -1
+    # meta update: n_new < 1, new_k without new_v
+    assert L.csa_meta_update(ctypes.byref(d), *P[:5], None, None, 0, FAKE, 1 << 40, None) == -1
+    assert L.csa_meta_update(ctypes.byref(d), *P[:5], FAKE, None, 1, FAKE, 1 << 40, None) == -1
+    # status read without a workspace
+    assert L.csa_get_device_status(None, None, None) == -3
+
+
+def test_binding_requires_cuda_tensors():
+    import torch
+    d = dims(B=1, Hq=4, Hkv=1, max_pages_per_seq=4, num_pages=4, max_sel=4)
+    with pytest.raises(ValueError):
+        csa.decode_full(d, torch.zeros(1, 4, 128, dtype=torch.bfloat16), None, None, None, None,
+                        None, torch.zeros(8, dtype=torch.uint8))

@@ -1,0 +1,215 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs (metadata bit-exact, scores to fp32 accuracy, selection by
+the band rule, attention within max-abs 2e-2 / mean-abs 2e-3 of fp32)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_decoding_b200 import csa
+from long_context_decoding_b200 import workloads as wl
+from parity import (Run, assert_meta_equal, assert_out_close, assert_scores_close,
+                    check_selection)
+
+pytestmark = pytest.mark.gpu
+PS = 16
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    oracle.set_threads(0)
+    yield
+
+
+def full_check(run: Run, dense=True):
+    """meta -> score/select -> decode (on the oracle's selection) -> dense."""
+    meta = run.gpu_meta()
+    assert_meta_equal(run, meta)
+    ref = run.oracle_step()
+    scores = run.gpu_select()
+    torch.cuda.synchronize()
+    assert_scores_close(scores, ref["scores"])
+    check_selection(run.layer.sel, run.layer.n_sel, ref["scores"], ref["sel"], ref["nsel"],
+                    gpu_scores=scores)
+    # decode parity on the oracle's own selection (oracle -> CUDA only)
+    osel = torch.from_numpy(np.ascontiguousarray(ref["sel"])).to(run.c.q.device)
+    onsel = torch.from_numpy(ref["nsel"]).to(run.c.q.device)
+    if osel.shape[2] != run.d.max_sel:
+        pad = torch.full((run.d.B, run.d.Hkv, run.d.max_sel), -1, dtype=torch.int32,
+                         device=run.c.q.device)
+        pad[:, :, :osel.shape[2]] = osel
+        osel = pad
+    out, lse = run.gpu_decode(osel, onsel)
+    errs = {"sparse": assert_out_close(out, lse, ref["out"], ref["lse"], "sparse decode")}
+    assert csa.device_status(run.ws) == 0
+    if dense:
+        dout, dlse = run.gpu_dense()
+        rout, rlse = run.oracle_dense()
+        errs["dense"] = assert_out_close(dout, dlse, rout, rlse, "dense decode")
+        assert csa.device_status(run.ws) == 0
+    return errs
+
+
+@pytest.mark.parametrize("w", [wl.TINY, wl.CTX32K], ids=lambda w: w.name)
+def test_workload_parity(w, cuda):
+    run = Run(wl.make_case(w, cuda))
+    full_check(run)
+
+
+def test_workload_parity_64k_planted(cuda):
+    run = Run(wl.make_case(wl.CTX64K, cuda))
+    full_check(run)
+
+
+# ---------------------------------------------------------------- edge cases
+def small(B=2, Hq=8, Hkv=2, D=128, lens=(1000, 777), prefix=20, window=50, budget=160, seed=3,
+          extra=0):
+    return wl.Workload("edge", B=B, Hq=Hq, Hkv=Hkv, D=D, seq_lens=tuple(lens), prefix=prefix,
+                       window=window, budget=budget, seed=seed, steps=extra)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_group_sizes_and_head_dims(G, D, cuda):
+    w = small(Hq=2 * G, Hkv=2, D=D, lens=(900, 523))
+    full_check(Run(wl.make_case(w, cuda)))
+
+
+@pytest.mark.parametrize("lens,P,W,budget", [
+    ((1,), 0, 0, 16),            # one token
+    ((15,), 3, 4, 32),           # shorter than a page
+    ((16,), 0, 0, 0),            # exactly one page, nothing but prefix/window (empty)
+    ((300,), 0, 0, 64),          # no prefix, no window: pure top-k
+    ((300,), 17, 33, 0),         # budget 0: prefix + window only, ragged boundaries
+    ((300,), 40, 40, 10_000),    # budget covers everything -> dense
+    ((300,), 200, 150, 32),      # prefix + window cover everything
+    ((257, 1030, 48), 5, 7, 48), # ragged batch, boundary pages partial on both sides
+    ((4096 + 5,), 64, 256, 512), # ragged tail page
+    ((33,), 17, 15, 16),         # one candidate page partial on both sides
+])
+def test_edge_geometry(lens, P, W, budget, cuda):
+    w = small(B=len(lens), lens=lens, prefix=P, window=W, budget=budget)
+    full_check(Run(wl.make_case(w, cuda)))
+
+
+def test_empty_sequence_outputs_zero(cuda):
+    w = small(B=2, lens=(0, 100), prefix=4, window=8, budget=32)
+    run = Run(wl.make_case(w, cuda))
+    run.gpu_meta()
+    run.gpu_select()
+    out, lse = run.gpu_decode(run.layer.sel, run.layer.n_sel)
+    torch.cuda.synchronize()
+    assert (out[0].float() == 0).all() and torch.isneginf(lse[0]).all()
+    assert torch.isfinite(out[1].float()).all()
+    assert csa.device_status(run.ws) == 0
+
+
+def test_maximum_budget_and_long_candidate_list(cuda):
+    """16k+ candidate pages of one unit, k = 512."""
+    w = small(B=1, Hq=8, Hkv=1, D=128, lens=(262144 + 77,), prefix=128, window=512,
+              budget=8192)
+    run = Run(wl.make_case(w, cuda))
+    full_check(run, dense=False)
+
+
+def test_bad_page_id_sets_device_flag(cuda):
+    w = small(B=1, lens=(600,), prefix=16, window=32, budget=64)
+    case = wl.make_case(w, cuda)
+    run = Run(case)
+    run.gpu_meta()
+    assert csa.device_status(run.ws) == 0
+    case.page_table[0, 5] = w.num_pages + 7        # out of range
+    run.gpu_select()
+    out, lse = run.gpu_decode(run.layer.sel, run.layer.n_sel)
+    flags = csa.device_status(run.ws)
+    assert flags & csa.DEVFLAG_BAD_PAGE_ID
+    assert csa.device_status(run.ws) == 0           # cleared by the read
+
+
+def test_bad_selection_sets_device_flag(cuda):
+    w = small(B=1, lens=(600,), prefix=16, window=32, budget=64)
+    run = Run(wl.make_case(w, cuda))
+    run.gpu_meta()
+    run.gpu_select()
+    sel = run.layer.sel.clone()
+    sel[0, 0, 1] = sel[0, 0, 0]                     # not strictly ascending
+    run.gpu_decode(sel, run.layer.n_sel)
+    assert csa.device_status(run.ws) & csa.DEVFLAG_BAD_SELECTION
+
+
+# ---------------------------------------------------------------- append
+def test_incremental_append_matches_rebuild(cuda):
+    """64 single-token appends through csa_meta_update: cache slots hold the
+    new tokens and the incremental min/max equals the oracle's recomputation
+    on a host cache built by placing the same tokens."""
+    steps = 64
+    w = small(B=3, Hq=8, Hkv=2, D=128, lens=(1000, 1015, 1024), prefix=16, window=64,
+              budget=128, extra=steps)
+    case = wl.make_case(w, cuda)
+    run = Run(case)
+    run.gpu_meta()
+    host_k = run.h["k"].copy()
+    host_v = run.h["v"].copy()
+    pt = run.h["pt"]
+    lens = [int(x) for x in run.h["sl"]]
+    for step in range(steps):
+        q, nk, nv = wl.step_tokens(case, step)
+        for b in range(w.B):
+            t = lens[b]
+            host_k[pt[b, t // PS], :, t % PS] = wl.bits(nk[b, 0])
+            host_v[pt[b, t // PS], :, t % PS] = wl.bits(nv[b, 0])
+            lens[b] += 1
+        case.seq_lens += 1
+        csa.meta_update(run.d, case.k_cache, case.v_cache, run.layer.meta, case.page_table,
+                        case.seq_lens, nk, nv, 1, run.ws)
+    torch.cuda.synchronize()
+    assert csa.device_status(run.ws) == 0
+    run.h.update(k=host_k, v=host_v, sl=np.array(lens, np.int32))
+    # the cache: every appended slot holds the new token
+    gk, gv = wl.bits(case.k_cache), wl.bits(case.v_cache)
+    for b in range(w.B):
+        for t in range(lens[b] - steps, lens[b]):
+            phys, slot = pt[b, t // PS], t % PS
+            np.testing.assert_array_equal(gk[phys, :, slot], host_k[phys, :, slot])
+            np.testing.assert_array_equal(gv[phys, :, slot], host_v[phys, :, slot])
+    assert_meta_equal(run, run.layer.meta)
+
+
+def test_chunk_append_prefill(cuda):
+    """A multi-token chunk append (prefill of 333 tokens after 50)."""
+    w = small(B=2, Hq=4, Hkv=2, D=64, lens=(50, 50), prefix=8, window=16, budget=64, extra=333)
+    case = wl.make_case(w, cuda)
+    run = Run(case)
+    run.gpu_meta()
+    g = torch.Generator(device=cuda).manual_seed(5)
+    nk = torch.randn((w.B, 333, w.Hkv, w.D), generator=g, device=cuda).to(torch.bfloat16)
+    nv = torch.randn((w.B, 333, w.Hkv, w.D), generator=g, device=cuda).to(torch.bfloat16)
+    case.seq_lens += 333
+    csa.meta_update(run.d, case.k_cache, case.v_cache, run.layer.meta, case.page_table,
+                    case.seq_lens, nk, nv, 333, run.ws)
+    torch.cuda.synchronize()
+    host_k, pt = run.h["k"].copy(), run.h["pt"]
+    nkb = wl.bits(nk)
+    for b in range(w.B):
+        for i in range(333):
+            t = 50 + i
+            host_k[pt[b, t // PS], :, t % PS] = nkb[b, i]
+    run.h.update(k=host_k, sl=case.seq_lens.cpu().numpy())
+    assert_meta_equal(run, run.layer.meta)
+    assert csa.device_status(run.ws) == 0
+
+
+def test_repeat_calls_reuse_workspace(cuda):
+    """Tickets left at zero: the same workspace serves many calls."""
+    run = Run(wl.make_case(wl.TINY, cuda))
+    run.gpu_meta()
+    run.gpu_select()
+    out1, _ = run.gpu_decode(run.layer.sel, run.layer.n_sel)
+    for _ in range(5):
+        out2, _ = run.gpu_decode(run.layer.sel, run.layer.n_sel)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
