@@ -199,8 +199,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     }
     __syncthreads();
     const long long T = uoff[units];
-    const int n_cta = (int)gridDim.x;
-    const long long s = T * blockIdx.x / n_cta, e = T * (blockIdx.x + 1) / n_cta;
+    // partition over at most T CTAs so that every participating CTA owns at
+    // least one item: the merge counts every CTA between a unit's first and
+    // last one
+    const int n_cta = (int)(T < (long long)gridDim.x ? (T > 0 ? T : 1) : gridDim.x);
+    const long long s = blockIdx.x < (unsigned)n_cta ? T * blockIdx.x / n_cta : T;
+    const long long e = blockIdx.x < (unsigned)n_cta ? T * (blockIdx.x + 1) / n_cta : T;
 
     // units with nothing to attend (empty sequences): out = 0, lse = -inf
     if (blockIdx.x == 0) {
