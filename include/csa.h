@@ -187,6 +187,32 @@ int csa_decode_full(const csa_dims *d, const void *q, const void *k_cache,
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * csa_decode for callers that cannot allocate device memory.  The paper has
+ * no counterpart to this entry point; it exists for deployment: a plugin
+ * hosted inside another runtime that owns every device buffer, or a server
+ * that reserves all device memory at start-up and allows no allocation later,
+ * has no way to provide the workspace csa_decode needs.
+ *
+ * Same arguments, results and conventions as csa_decode, minus the
+ * workspace.  The split-K scratch lives in a 4 MiB __device__ array inside
+ * the library (held on every GPU that loads it until the process exits).
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine).  A shape whose scratch would exceed 4 MiB is rejected with
+ * CSA_ERR_WORKSPACE; at D = 128, G = 8 on a 148-SM B200 that is about
+ * 700 (sequence, kv-head) units.  The first call on a device looks up the
+ * array's device address (make it before any stream capture).  The call
+ * clears the array's flag word and tickets on `stream` before the kernel;
+ * every call shares the array, so calls that overlap on the GPU race: keep
+ * them on one stream or otherwise ordered.  Device-side flags of this call
+ * are not reported (offending pages are still skipped).
+ */
+int csa_decode_noalloc(const csa_dims *d, const void *q, const void *k_cache,
+                       const void *v_cache, const int32_t *page_table,
+                       const int32_t *seq_lens, const int32_t *sel_pages,
+                       const int32_t *n_sel, int prefix, int window, float scale,
+                       void *out, float *lse, void *stream);
+
+/*
  * Synchronise `stream`, read and clear the device flag word of `workspace`.
  * Returns CSA_OK when no flag was set, CSA_ERR_DEVICE_FLAG when one was (the
  * CSA_DEVFLAG_* bits go to *flags_out if it is not NULL), CSA_ERR_CUDA on a

@@ -26,7 +26,7 @@ DEVFLAG_TIMEOUT = 8
 
 EXPORTS = ("csa_version", "csa_status_string", "csa_workspace_size", "csa_workspace_init",
            "csa_meta_update", "csa_score_select", "csa_decode", "csa_decode_full",
-           "csa_get_device_status")
+           "csa_get_device_status", "csa_decode_noalloc")
 
 
 class CsaError(RuntimeError):
@@ -168,6 +168,28 @@ def decode_full(d: Dims, q, k_cache, v_cache, page_table, seq_lens, out, ws, lse
         _ptr(v_cache, bf, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
         _ptr(seq_lens, torch.int32, "seq_lens"), float(scale), _ptr(out, bf, "out"),
         _ptr(lse, torch.float32, "lse"), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def decode_noalloc(d: Dims, q, k_cache, v_cache, page_table, seq_lens, sel, n_sel, prefix: int,
+                   window: int, out, lse=None, scale: float = 0.0, stream=None):
+    """csa_decode without a workspace, for callers that cannot allocate device
+    memory (a plugin inside a runtime that owns all device buffers, a server
+    that reserves the GPU at start-up): the scratch is a fixed 4 MiB array
+    inside the library, shared by every call on the device, so calls must
+    not overlap on the GPU.  Device-side flags of this call are not
+    reported."""
+    f = lib().csa_decode_noalloc
+    P = ctypes.c_void_p
+    f.argtypes = [ctypes.POINTER(Dims), P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_float, P, P, P]
+    f.restype = ctypes.c_int
+    bf = torch.bfloat16
+    _check("csa_decode_noalloc", f(
+        ctypes.byref(d), _ptr(q, bf, "q"), _ptr(k_cache, bf, "k_cache"),
+        _ptr(v_cache, bf, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(sel, torch.int32, "sel"),
+        _ptr(n_sel, torch.int32, "n_sel"), int(prefix), int(window), float(scale),
+        _ptr(out, bf, "out"), _ptr(lse, torch.float32, "lse"), _stream(stream)))
 
 
 def device_status(ws, stream=None) -> int:

@@ -1,0 +1,176 @@
+// noalloc.cu -- csa_decode_noalloc: the sparse decode of csa_decode with its
+// scratch memory built into the library.
+//
+// Some callers cannot allocate device memory at all: a plugin hosted inside
+// another runtime that owns every device buffer and hands the plugin only
+// its inputs and outputs, or a serving process that reserves the whole GPU
+// for its KV cache at start-up and forbids any allocation afterwards.  Such a
+// caller cannot provide the workspace csa_decode needs for its split-K
+// partial results.  This entry point runs the same decode kernel, but its
+// scratch (flag word, merge tickets and partial records) lives in one
+// file-scope __device__ array of kNoAllocScratchBytes that every GPU which
+// loads the library keeps until the process exits.  The call itself
+// allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+//
+// The host name of that array is only a stand-in; the kernels get its device
+// address, looked up once per device (with that device current) through
+// cudaGetSymbolAddress on the first call made on the device.  Make that first
+// call before any stream capture.
+//
+// All calls share the one array and it keeps whatever the previous call left:
+// the flag word and the tickets are cleared on the caller's stream at the
+// start of every call; the partial records need no clearing.  Two calls whose
+// kernels overlap on a GPU therefore race on the array: issue them on one
+// stream, or order them.
+#include <math.h>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace csa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;   // 4 MiB per GPU
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mu;
+
+// Device address of g_noalloc_scratch on the current device (nullptr on error).
+void* scratch_address(int dev) {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_scratch_addr[dev] = p;
+    }
+    return g_scratch_addr[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Same view of a paged cache as csa_decode uses: [num_pages * Hkv * 16][D]
+// bf16, 64-channel x 16-token boxes, 128-byte swizzle.
+bool cache_map(CUtensorMap* m, const void* base, const Shape& s) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)s.D, (cuuint64_t)s.NPG * s.Hkv * kPage};
+    cuuint64_t strides[1] = {(cuuint64_t)s.D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kPage};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+bool ok16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" int csa_decode_noalloc(const csa_dims* d, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* page_table,
+                                  const int32_t* seq_lens, const int32_t* sel_pages,
+                                  const int32_t* n_sel, int prefix, int window, float scale,
+                                  void* out, float* lse, void* stream) {
+    if (!d || d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->max_pages_per_seq < 1 ||
+        d->num_pages < 1 || d->max_sel < 1 || d->Hq % d->Hkv != 0)
+        return CSA_ERR_INVALID_ARG;
+    const int G = d->Hq / d->Hkv;
+    if (d->page_size != kPage || (d->D != 64 && d->D != 128 && d->D != 256) ||
+        (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) ||
+        (long long)d->B * d->Hkv > kMaxUnits ||
+        (long long)d->num_pages * d->Hkv * kPage >= (1ll << 31) ||
+        (long long)d->max_pages_per_seq * kPage >= (1ll << 31))
+        return CSA_ERR_UNSUPPORTED;
+    if (!ok16(q) || !ok16(k_cache) || !ok16(v_cache) || !ok16(page_table) || !ok16(seq_lens) ||
+        !ok16(sel_pages) || !ok16(n_sel) || !ok16(out) || (lse && !ok16(lse)))
+        return CSA_ERR_INVALID_ARG;
+    if (prefix < 0 || window < 0 || !(scale == scale) || isinf(scale)) return CSA_ERR_INVALID_ARG;
+
+    Shape s;
+    s.B = d->B;
+    s.Hq = d->Hq;
+    s.Hkv = d->Hkv;
+    s.G = G;
+    s.D = d->D;
+    s.MP = d->max_pages_per_seq;
+    s.NPG = d->num_pages;
+    s.max_sel = d->max_sel;
+
+    // scratch: [flag word | tickets | partial records], each 256-byte aligned
+    const size_t units = (size_t)s.B * s.Hkv;
+    const size_t tickets_off = 256;
+    const size_t partials_off = tickets_off + up256(4 * units);
+    const size_t slots = (size_t)decode_grid(s) + units;
+    const size_t need = partials_off + 4 * slots * (size_t)G * (s.D + 2);
+    if (need > kNoAllocScratchBytes) return CSA_ERR_WORKSPACE;   // shape needs more scratch
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    uint8_t* scratch = static_cast<uint8_t*>(scratch_address(dev));
+    if (!scratch) return CSA_ERR_CUDA;
+
+    CUtensorMap tmK, tmV;
+    if (!cache_map(&tmK, k_cache, s) || !cache_map(&tmV, v_cache, s)) return CSA_ERR_CUDA;
+
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(scratch, 0, partials_off, st) != cudaSuccess) {   // flag + tickets
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    DecodeParams p;
+    p.q = static_cast<const uint16_t*>(q);
+    p.page_table = page_table;
+    p.seq_lens = seq_lens;
+    p.sel = sel_pages;
+    p.n_sel = n_sel;
+    p.prefix = prefix;
+    p.window = window;
+    p.dense = 0;
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)s.D);
+    p.scale_log2 = sc * 1.4426950408889634f;
+    p.out = static_cast<uint16_t*>(out);
+    p.lse = lse;
+    p.flags = reinterpret_cast<uint32_t*>(scratch);
+    p.tickets = reinterpret_cast<uint32_t*>(scratch + tickets_off);
+    p.partials = reinterpret_cast<float*>(scratch + partials_off);
+    p.s = s;
+    if (launch_decode(p, tmK, tmV, st) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    return CSA_OK;
+}
