@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--profile", action="store_true",
                     help="timed steps only (for an ncu launch list): no baseline, e2e, clocks")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="use only the first N layers (small cases for ncu captures)")
     return ap.parse_args()
 
 
@@ -495,6 +497,8 @@ def main():
     args = parse_args()
     dist = Dist()
     base = wl.CTX256K if args.workload == "ctx256k" else replace(wl.CTX64K, steps=0)
+    if args.layers:
+        base = replace(base, layers=args.layers)
     try:
         if args.impl == "reference":
             run_reference(args, dist, base)
