@@ -14,6 +14,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/csa.h"
 
 namespace csa {
@@ -206,6 +208,28 @@ __host__ __device__ __forceinline__ SeqGeom seq_geom(int L, int prefix, int wind
         s.c_hi = 0;
     }
     return s;
+}
+
+// ------------------------------------------------------------ launches
+// Launch with programmatic stream serialization: the grid may start while
+// the previous kernel on the stream is still running.  Every kernel of this
+// library therefore reads only caller inputs before pdl_wait(), and calls
+// pdl_launch_dependents() only after it, so that when a kernel starts, all
+// kernels two or more launches earlier have completed.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace csa

@@ -106,6 +106,8 @@ static int check_dims(const csa_dims* d, Shape* s) {
     if ((long long)d->B * d->Hkv > kMaxUnits) return CSA_ERR_UNSUPPORTED;
     if ((long long)d->num_pages * d->Hkv * kPage >= (1ll << 31)) return CSA_ERR_UNSUPPORTED;
     if ((long long)d->max_pages_per_seq * kPage >= (1ll << 31)) return CSA_ERR_UNSUPPORTED;
+    if ((long long)d->B * d->Hkv * (d->max_pages_per_seq + 2) >= (1ll << 31))
+        return CSA_ERR_UNSUPPORTED;   // flattened page lists are indexed with int
     s->B = d->B;
     s->Hq = d->Hq;
     s->Hkv = d->Hkv;
@@ -256,7 +258,6 @@ int csa_score_select(const csa_dims* d, const void* q, const void* meta,
     lp.sel = sel_pages;
     lp.n_sel = n_sel;
     lp.flags = sp.flags;
-    lp.smem_keys = 0;
     lp.s = s;
     return launch_status(launch_select(lp, st));
 }

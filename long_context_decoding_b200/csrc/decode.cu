@@ -45,7 +45,10 @@ struct DecCfg {
     static constexpr int kBoxes = D / 64;               // 64-channel TMA boxes per K (or V) page
     static constexpr int kHalf = kBoxes * 2048;         // bytes of one page's K (or V) tile
     static constexpr int kStageBytes = 2 * kHalf;
-    static constexpr int kStages = D == 256 ? 4 : (D == 128 ? 9 : 16);
+    static constexpr int kStages = D == 256 ? 4 : (D == 128 ? 8 : 16);
+    // a stage's previous use must belong to the same consumer warp, so that a
+    // parity wait can never be two phases ahead of the barrier
+    static_assert(kStages % kConsumers == 0, "stages must be a multiple of consumers");
     static constexpr int kHeads = 8 * NB;               // query heads per CTA (padded)
     static constexpr int kMB = D / 16;                  // 16-channel blocks
     static constexpr size_t kOw = (size_t)kConsumers * kHeads * D * 4;
@@ -53,7 +56,11 @@ struct DecCfg {
     static constexpr size_t kItems = (size_t)kDecodeItemCap * 8;
     static __host__ __device__ size_t smem_bytes(int units) {
         return 1024 /* alignment slack */ + (size_t)kStages * kStageBytes + kOw + kMl + kItems +
-               (((size_t)(units + 1) * 4 + 15) & ~(size_t)15) + 16 * (size_t)kStages;
+               unit_bytes(units) + 16 * (size_t)kStages;
+    }
+    // uoff [units + 1] | uinfo [units] (int2: seq_len, n_sel | n_blo << 30 | n_bhi << 31)
+    static __host__ __device__ size_t unit_bytes(int units) {
+        return (((size_t)(units + 1) * 4 + 15) & ~(size_t)15) + (size_t)units * 8;
     }
 };
 
@@ -107,6 +114,33 @@ __device__ UnitPlan make_plan(const DecodeParams& p, int u) {
     return q;
 }
 
+// The plan of unit u again, from the (seq_len, packed counts) kept in
+// shared memory by the first pass: no global loads.
+__device__ __forceinline__ UnitPlan cached_plan(const DecodeParams& p, int u, int2 info) {
+    UnitPlan q;
+    q.b = u / p.s.Hkv;
+    q.g = u % p.s.Hkv;
+    const SeqGeom sg = seq_geom(info.x, p.prefix, p.window);
+    q.L = info.x;
+    q.Pe = sg.Pe;
+    q.We = sg.We;
+    q.np = sg.np;
+    q.c_lo = sg.c_lo;
+    q.c_hi = sg.c_hi;
+    q.n_sel = info.y & 0x3fffffff;
+    q.n_blo = (info.y >> 30) & 1;
+    q.n_bhi = (int)(((unsigned)info.y >> 31) & 1u);
+    q.sel = p.sel ? p.sel + (size_t)u * p.s.max_sel : nullptr;
+    if (p.dense || sg.c_lo == sg.c_hi) {
+        q.n_pre = sg.np;
+        q.n_win = 0;
+    } else {
+        q.n_pre = sg.c_lo;
+        q.n_win = sg.np - sg.c_hi;
+    }
+    return q;
+}
+
 // Item j of a unit's list -> logical page and whether all its valid tokens
 // are attended (else the prefix/window token mask applies).  Returns false
 // for a selection entry that is out of range or out of order.
@@ -151,6 +185,84 @@ __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(4 * 32) : "memory");
 }
 
+// The CTA holding a unit's last ticket merges the unit's partial records
+// (o relative to its own max m, with m and l) written by CTAs
+// first .. last:  M = max_r m_r,  w_r = 2^(m_r - M),  out = sum_r w_r o_r /
+// sum_r w_r l_r.  Records are read through L2 in chunks: the weights of a
+// chunk go to shared memory first, then every thread sums its (head, channel)
+// elements with independent loads.
+template <int D>
+__device__ void merge_records(const DecodeParams& p, int b, int g, int u, int first, int last,
+                              size_t rec_stride, float* wsm, float* Msm, float* Lsm, int ctid) {
+    const int G = p.s.G, Hq = p.s.Hq;
+    const int nrec = last - first + 1;
+    const float* base = p.partials + ((size_t)first + u) * rec_stride;
+    // M and L per head: one warp per head, lanes over records
+    const int warp = ctid >> 5, lane = ctid & 31;
+    for (int h = warp; h < G; h += 4) {
+        float m = -INFINITY;
+        for (int r = lane; r < nrec; r += 32)
+            m = fmaxf(m, __ldcg(base + (size_t)r * rec_stride + (size_t)h * (D + 2) + D));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float l = 0.f;
+        for (int r = lane; r < nrec; r += 32) {
+            const float* rc = base + (size_t)r * rec_stride + (size_t)h * (D + 2);
+            const float mr = __ldcg(rc + D);
+            l += mr == -INFINITY ? 0.f : __ldcg(rc + D + 1) * ex2(mr - m);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) {
+            Msm[h] = m;
+            Lsm[h] = l;
+        }
+    }
+    consumer_sync();
+    constexpr int kPer = 8;                       // elements per thread and pass
+    const int total = G * D;
+    const int chunk = (4 * 8 * D) / G;            // records whose weights fit in wsm
+    for (int e0 = 0; e0 < total; e0 += 128 * kPer) {
+        float acc[kPer];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
+        for (int r0 = 0; r0 < nrec; r0 += chunk) {
+            const int rn = nrec - r0 < chunk ? nrec - r0 : chunk;
+            for (int i = ctid; i < rn * G; i += 128) {
+                const int r = r0 + i / G, h = i % G;
+                const float mr = __ldcg(base + (size_t)r * rec_stride + (size_t)h * (D + 2) + D);
+                wsm[i] = mr == -INFINITY ? 0.f : ex2(mr - Msm[h]);
+            }
+            consumer_sync();
+            for (int r = 0; r < rn; ++r) {
+                const float* rc = base + (size_t)(r0 + r) * rec_stride;
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) {
+                    const int idx = e0 + j * 128 + ctid;
+                    if (idx < total) {
+                        const int h = idx / D, c = idx % D;
+                        acc[j] += __ldcg(rc + (size_t)h * (D + 2) + c) * wsm[r * G + h];
+                    }
+                }
+            }
+            consumer_sync();
+        }
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int idx = e0 + j * 128 + ctid;
+            if (idx < total) {
+                const int h = idx / D, c = idx % D;
+                const float l = Lsm[h];
+                const size_t oi = (size_t)b * Hq + (size_t)g * G + h;
+                p.out[oi * D + c] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(l > 0.f ? acc[j] / l : 0.f));
+                if (c == 0 && p.lse)
+                    p.lse[oi] = l > 0.f ? (Msm[h] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+            }
+        }
+    }
+}
+
 template <int D, int NB>
 __global__ void __launch_bounds__(DecCfg<D, NB>::kThreads)
 decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -166,16 +278,29 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     int2* items = reinterpret_cast<int2*>(ls + C::kConsumers * C::kHeads);
     int* uoff = reinterpret_cast<int*>(items + kDecodeItemCap);
     const int units = p.s.B * p.s.Hkv;
-    uint64_t* full = reinterpret_cast<uint64_t*>(
-        reinterpret_cast<uint8_t*>(uoff) + (((size_t)(units + 1) * 4 + 15) & ~(size_t)15));
+    int2* uinfo = reinterpret_cast<int2*>(reinterpret_cast<uint8_t*>(uoff) +
+                                          (((size_t)(units + 1) * 4 + 15) & ~(size_t)15));
+    uint64_t* full = reinterpret_cast<uint64_t*>(uinfo + units);
     uint64_t* empty = full + C::kStages;
     __shared__ int s_abort, s_last, s_issued;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Hkv = p.s.Hkv, G = p.s.G, Hq = p.s.Hq;
+    if (tid == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    // the selection, the appended tokens and the previous users of the
+    // workspace belong to earlier kernels
+    pdl_wait();
+    pdl_launch_dependents();
 
     // ---- per-unit list lengths and their exclusive scan
-    for (int u = tid; u < units; u += C::kThreads) uoff[u] = make_plan(p, u).total();
+    for (int u = tid; u < units; u += C::kThreads) {
+        const UnitPlan q = make_plan(p, u);
+        uoff[u] = q.total();
+        uinfo[u] = make_int2(q.L, q.n_sel | (q.n_blo << 30) | (q.n_bhi << 31));
+    }
     if (tid == 0) {
         s_abort = 0;
         s_issued = 0;
@@ -223,7 +348,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     // ---- resolve the physical page of every item of this CTA's slice
     for (long long x = s + tid; x < e; x += C::kThreads) {
         const int u = find_unit(uoff, units, x);
-        const UnitPlan q = make_plan(p, u);
+        const UnitPlan q = cached_plan(p, u, uinfo[u]);
         int page = 0;
         bool whole = true;
         int phys = -1;
@@ -500,28 +625,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 consumer_sync();
                 if (s_last) {
                     __threadfence();
-                    for (int idx = ctid; idx < G * D; idx += 128) {
-                        const int h = idx / D, c = idx % D;
-                        float M = -INFINITY;
-                        for (int ci = first_cta; ci <= last_cta; ++ci)
-                            M = fmaxf(M, __ldcg(p.partials + ((size_t)ci + u) * rec_stride +
-                                                (size_t)h * (D + 2) + D));
-                        float acc = 0.f, lsum = 0.f;
-                        for (int ci = first_cta; ci <= last_cta; ++ci) {
-                            const float* rc = p.partials + ((size_t)ci + u) * rec_stride +
-                                              (size_t)h * (D + 2);
-                            const float mc = __ldcg(rc + D);
-                            const float f = mc == -INFINITY ? 0.f : ex2(mc - M);
-                            acc += __ldcg(rc + c) * f;
-                            lsum += __ldcg(rc + D + 1) * f;
-                        }
-                        const size_t oi = ((size_t)b * Hq + (size_t)g * G + h);
-                        const float val = lsum > 0.f ? acc / lsum : 0.f;
-                        p.out[oi * D + c] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
-                        if (c == 0 && p.lse)
-                            p.lse[oi] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f
-                                                   : -INFINITY;
-                    }
+                    merge_records<D>(p, b, g, u, first_cta, last_cta, rec_stride, Ow, ms, ls,
+                                     ctid);
                     if (ctid == 0) atomicExch(&p.tickets[u], 0u);
                 }
             }
@@ -555,8 +660,7 @@ cudaError_t launch_decode_t(const DecodeParams& p, const CUtensorMap& tmK, const
         attr_done[dev] = 1;
     }
     const int grid = decode_grid(p.s);
-    decode_kernel<D, NB><<<grid, C::kThreads, smem, st>>>(tmK, tmV, p);
-    return cudaGetLastError();
+    return launch_pdl(decode_kernel<D, NB>, dim3(grid), dim3(C::kThreads), smem, st, tmK, tmV, p);
 }
 
 }  // namespace

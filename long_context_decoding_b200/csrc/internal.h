@@ -61,7 +61,6 @@ struct SelectParams {
     int32_t* sel;
     int32_t* n_sel;
     uint32_t* flags;
-    int smem_keys;          // set by the launcher
     Shape s;
 };
 cudaError_t launch_select(const SelectParams& p, cudaStream_t st);

@@ -94,6 +94,8 @@ __device__ void update_page(const MetaParams& p, int b, int g, int c, int L, int
 }
 
 __global__ void meta_update_kernel(MetaParams p) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int u = blockIdx.x;
     const int Hkv = p.s.Hkv, D = p.s.D, MP = p.s.MP;
     const int b = u / Hkv, g = u % Hkv;
@@ -120,8 +122,7 @@ cudaError_t launch_meta_update(const MetaParams& p, cudaStream_t st) {
     if (pages > 65535) pages = 65535;                       // grid.y limit; the kernel strides
     if (units == 0 || pages <= 0) return cudaSuccess;
     dim3 grid(units, pages);
-    meta_update_kernel<<<grid, p.s.D / 2, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(meta_update_kernel, grid, dim3(p.s.D / 2), 0, st, p);
 }
 
 }  // namespace csa

@@ -37,7 +37,10 @@ struct ScoreCfg {
     static constexpr int kRowBytes = 4 * D;           // [min | max] bf16 of one (page, kv-head)
     static constexpr int kRowStride = 4 * D + 16;     // padded shared-memory row
     static constexpr int kStageBytes = kTile * kRowStride;
-    static constexpr int kStages = D >= 256 ? 5 : 8;
+    static constexpr int kStages = D >= 256 ? 4 : 8;
+    // a stage's previous use must belong to the same consumer warp, so that a
+    // parity wait can never be two phases ahead of the barrier
+    static_assert(kStages % kConsumers == 0, "stages must be a multiple of consumers");
     static constexpr int kKPairs = 2 * D / 32;        // 32-channel steps along [min | max]
     // stages | page-table slice | full/empty barriers | tile infos | 3 x [B + 1] ints
     static __host__ __device__ size_t smem_bytes(int B) {
@@ -67,27 +70,52 @@ __device__ __forceinline__ uint32_t pos_part(uint32_t w) {   // max(q, 0) per bf
 }
 
 // Walks the CTA's range [x, e) of the flattened candidate list in tiles that
-// never cross a (sequence, kv-head) unit.
+// never cross a (sequence, kv-head) unit.  One division at start-up; every
+// step after that is a few integer adds.
 struct TileWalker {
-    long long x, e;
+    int x, e;
     const int* seq_off;   // [B + 1]: first flattened index of sequence b
     const int* seq_n;     // candidates per (b, kv-head)
-    const int* seq_clo;
-    int Hkv, b;
-    __device__ bool next(TileInfo& t) {
+    const int* seq_clo;   // first candidate page of sequence b
+    int Hkv, B;
+    int b, g, idx;        // unit and candidate index of position x
+
+    __device__ void start(int s, int end) {
+        x = s;
+        e = end;
+        int lo = 0, hi = B;                   // last b with seq_off[b] <= x
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (seq_off[mid] <= x) lo = mid; else hi = mid;
+        }
+        b = lo;
+        while (b < B - 1 && seq_n[b] == 0) ++b;
+        const int n = seq_n[b] > 0 ? seq_n[b] : 1;
+        const int rel = x - seq_off[b];
+        g = rel / n;
+        idx = rel - g * n;
+    }
+    // Next run of up to `cap` candidates inside one unit.
+    __device__ bool next(TileInfo& t, int cap = 16) {
         if (x >= e) return false;
-        while (x >= seq_off[b + 1]) ++b;
         const int n = seq_n[b];
-        const long long rel = x - seq_off[b];
-        const int g = (int)(rel / n), idx = (int)(rel % n);
-        long long end = seq_off[b] + (long long)(g + 1) * n;
-        if (end > e) end = e;
-        int cnt = (int)(end - x);
-        if (cnt > 16) cnt = 16;
+        int cnt = n - idx;
+        if (cnt > cap) cnt = cap;
+        if (cnt > e - x) cnt = e - x;
         t.unit = b * Hkv + g;
         t.first = seq_clo[b] + idx;
         t.count = cnt;
         x += cnt;
+        idx += cnt;
+        if (idx == n) {
+            idx = 0;
+            if (++g == Hkv) {
+                g = 0;
+                do {
+                    ++b;
+                } while (b < B && seq_n[b] == 0);
+            }
+        }
         return true;
     }
 };
@@ -247,32 +275,44 @@ score_kernel(ScoreParams p) {
     __syncthreads();
     const long long N = seq_off[B];
     const long long s = N * blockIdx.x / gridDim.x, e = N * (blockIdx.x + 1) / gridDim.x;
-    if (s >= e) return;
-
-    // Page-table slice of this CTA (the grid is sized so that e - s <= cap).
-    for (long long x = s + tid; x < e; x += C::kThreads) {
-        int b = 0, lo = 0, hi = B;            // last b with seq_off[b] <= x
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (seq_off[mid] <= x) lo = mid; else hi = mid;
-        }
-        b = lo;
-        const int n = seq_n[b];
-        const int idx = (int)((x - seq_off[b]) % n);
-        pt[x - s] = p.page_table[(size_t)b * MP + seq_clo[b] + idx];
+    if (s >= e) {
+        pdl_wait();
+        pdl_launch_dependents();
+        return;
     }
+
+    // Page-table slice of this CTA (the grid is sized so that e - s <= cap),
+    // copied run by run: every run is a contiguous piece of one page-table row.
+    TileWalker walk;
+    walk.seq_off = seq_off;
+    walk.seq_n = seq_n;
+    walk.seq_clo = seq_clo;
+    walk.Hkv = Hkv;
+    walk.B = B;
+    {
+        TileWalker fill = walk;
+        fill.start((int)s, (int)e);
+        TileInfo run;
+        int at = 0;
+        while (fill.next(run, 1 << 30)) {
+            const int32_t* src = p.page_table + (size_t)(run.unit / Hkv) * MP + run.first;
+            for (int i = tid; i < run.count; i += C::kThreads) pt[at + i] = __ldg(src + i);
+            at += run.count;
+        }
+    }
+    walk.start((int)s, (int)e);
+    __shared__ int s_issued;
     if (tid == 0) {
         for (int i = 0; i < C::kStages; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
         fence_barrier_init();
+        s_issued = 0;
     }
-    __syncthreads();
-
-    TileWalker walk{s, e, seq_off, seq_n, seq_clo, Hkv, 0};
-    __shared__ int s_issued;
-    if (tid == 0) s_issued = 0;
+    // the metadata was written by the previous kernel on the stream
+    pdl_wait();
+    pdl_launch_dependents();
     __syncthreads();
 
     if (warp == C::kConsumers) {
@@ -288,7 +328,7 @@ score_kernel(ScoreParams p) {
             __syncwarp();
             if (*(volatile int*)&s_abort) break;
             const int g = t.unit % Hkv;
-            const long long x0 = walk.x - t.count - s;   // slice index of row 0
+            const int x0 = walk.x - t.count - (int)s;    // slice index of row 0
             int phys = -1;
             bool ok = false;
             if (lane < t.count) {
@@ -340,8 +380,7 @@ cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t st) {
     const long long need = (ub + kScorePtCap - 1) / kScorePtCap;
     if (need > grid) grid = need;
     if (grid < 1) grid = 1;
-    score_kernel<D, NB><<<(unsigned)grid, C::kThreads, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(score_kernel<D, NB>, dim3((unsigned)grid), dim3(C::kThreads), smem, st, p);
 }
 
 }  // namespace

@@ -38,6 +38,7 @@ __device__ __forceinline__ uint32_t block_reduce_min_max(uint32_t v_min, uint32_
     return r;
 }
 
+template <bool kSmemKeys>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectParams p) {
     extern __shared__ __align__(16) uint32_t skeys[];
     __shared__ uint32_t hist[256];
@@ -55,6 +56,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectParams p) {
     const int n = sg.c_hi - sg.c_lo;
     const int kk = p.k_pages < n ? p.k_pages : n;
     int32_t* out = p.sel + (size_t)u * p.s.max_sel;
+    // scores (and the previous readers of sel) belong to earlier kernels
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (kk == n) {                              // every candidate fits the budget
         for (int i = tid; i < n; i += kSelThreads) out[i] = sg.c_lo + i;
@@ -66,16 +70,29 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectParams p) {
         return;
     }
 
-    // keys: shared memory when they fit, else in place over the fp32 scores
+    // keys: shared memory when they fit, else in place over the fp32 scores;
+    // eight independent loads per thread are in flight before any key is stored
     const float* sc = p.scores_ws + (size_t)u * MP + sg.c_lo;
-    uint32_t* keys = n <= p.smem_keys ? skeys : reinterpret_cast<uint32_t*>(
-                                                    p.scores_ws + (size_t)u * MP + sg.c_lo);
+    uint32_t* keys = kSmemKeys ? skeys : reinterpret_cast<uint32_t*>(
+                                             p.scores_ws + (size_t)u * MP + sg.c_lo);
     uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int i = tid; i < n; i += kSelThreads) {
-        const uint32_t k = order_key(sc[i]);
-        keys[i] = k;
-        kmin = min(kmin, k);
-        kmax = max(kmax, k);
+    for (int base = 0; base < n; base += 8 * kSelThreads) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + j * kSelThreads + tid;
+            v[j] = i < n ? __ldcg(sc + i) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + j * kSelThreads + tid;
+            if (i < n) {
+                const uint32_t k = order_key(v[j]);
+                keys[i] = k;
+                kmin = min(kmin, k);
+                kmax = max(kmax, k);
+            }
+        }
     }
     kmin = block_reduce_min_max(kmin, kmax, red, false);   // syncs also publish keys[]
     kmax = block_reduce_min_max(kmin, kmax, red, true);
@@ -192,7 +209,7 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t st) {
     cudaGetDevice(&dev);
     const int smem = kSmemKeys * 4;
     if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(select_kernel,
+        cudaError_t e = cudaFuncSetAttribute(select_kernel<true>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_done[dev] = 1;
@@ -201,10 +218,11 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t st) {
     if (units == 0) return cudaSuccess;
     // only as much shared memory as the longest candidate list needs; longer
     // lists keep their keys in place of the scores in global memory
-    SelectParams q = p;
-    q.smem_keys = p.s.MP <= kSmemKeys ? p.s.MP : 0;
-    select_kernel<<<units, kSelThreads, (size_t)q.smem_keys * 4, st>>>(q);
-    return cudaGetLastError();
+    if (p.s.MP <= kSmemKeys) {
+        return launch_pdl(select_kernel<true>, dim3(units), dim3(kSelThreads),
+                          (size_t)p.s.MP * 4, st, p);
+    }
+    return launch_pdl(select_kernel<false>, dim3(units), dim3(kSelThreads), 0, st, p);
 }
 
 }  // namespace csa
