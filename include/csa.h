@@ -105,13 +105,13 @@ typedef struct csa_dims {
 
 /* Bytes of device workspace the calls below need for shape *d (host
  * pointer).  Returns 0 for an invalid or unsupported shape.  The workspace
- * holds the device flag word, per-(sequence, kv-head) tickets, the fp32
+ * holds the device flag word, per-(sequence, kv-head) bookkeeping, the fp32
  * page scores and the split-K partial results. */
 size_t csa_workspace_size(const csa_dims *d);
 
 /* Zero `bytes` of `workspace` on `stream`.  Required once before the first
- * call that uses a fresh workspace; the kernels leave their tickets at zero
- * again when they finish. */
+ * call that uses a fresh workspace (the device flag word must start at
+ * zero). */
 int csa_workspace_init(void *workspace, size_t bytes, void *stream);
 
 /*
@@ -201,7 +201,7 @@ int csa_decode_full(const csa_dims *d, const void *q, const void *k_cache,
  * CSA_ERR_WORKSPACE; at D = 128, G = 8 on a 148-SM B200 that is about
  * 700 (sequence, kv-head) units.  The first call on a device looks up the
  * array's device address (make it before any stream capture).  The call
- * clears the array's flag word and tickets on `stream` before the kernel;
+ * clears the array's flag word on `stream` before the kernels;
  * every call shares the array, so calls that overlap on the GPU race: keep
  * them on one stream or otherwise ordered.  Device-side flags of this call
  * are not reported (offending pages are still skipped).

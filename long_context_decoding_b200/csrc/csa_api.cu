@@ -41,53 +41,15 @@ WsLayout workspace_layout(const Shape& s) {
     off = align_up(off + 4, 256);
     w.score_tickets = off;
     off = align_up(off + 4 * units, 256);
-    w.dec_tickets = off;
-    off = align_up(off + 4 * units, 256);
+    w.rec_range = off;
+    off = align_up(off + 8 * units, 256);
     w.scores = off;
     off = align_up(off + 4 * units * (size_t)s.MP, 256);
     w.partials = off;
     w.dec_slots = (size_t)decode_grid(s) + units;
-    off = align_up(off + 4 * w.dec_slots * (size_t)s.G * (s.D + 2), 256);
+    off = align_up(off + 4 * w.dec_slots * decode_record_floats(s), 256);
     w.total = off;
     return w;
-}
-
-// ---------------------------------------------------------------- tensor maps
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-        else
-            cudaGetLastError();
-    });
-    return fn;
-}
-
-// A [num_pages * Hkv * 16][D] bf16 view of a paged cache; boxes of
-// 64 channels x 16 tokens (one page of one kv-head, half or quarter of D),
-// 128-byte swizzle.
-static bool make_cache_map(CUtensorMap* m, const void* base, const Shape& s) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)s.D, (cuuint64_t)s.NPG * s.Hkv * kPage};
-    cuuint64_t strides[1] = {(cuuint64_t)s.D * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kPage};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 // ---------------------------------------------------------------- validation
@@ -258,6 +220,7 @@ int csa_score_select(const csa_dims* d, const void* q, const void* meta,
     lp.sel = sel_pages;
     lp.n_sel = n_sel;
     lp.flags = sp.flags;
+    lp.smem_keys = 0;
     lp.s = s;
     return launch_status(launch_select(lp, st));
 }
@@ -286,11 +249,10 @@ static int decode_common(const csa_dims* d, const void* q, const void* k_cache,
     WsLayout w;
     rc = check_ws(s, workspace, workspace_bytes, &w);
     if (rc != CSA_OK) return rc;
-    CUtensorMap tmK, tmV;
-    if (!make_cache_map(&tmK, k_cache, s) || !make_cache_map(&tmV, v_cache, s))
-        return CSA_ERR_CUDA;
     DecodeParams p;
     p.q = static_cast<const uint16_t*>(q);
+    p.k_cache = static_cast<const uint16_t*>(k_cache);
+    p.v_cache = static_cast<const uint16_t*>(v_cache);
     p.page_table = page_table;
     p.seq_lens = seq_lens;
     p.sel = sel_pages;
@@ -303,10 +265,10 @@ static int decode_common(const csa_dims* d, const void* q, const void* k_cache,
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
     p.flags = at<uint32_t>(workspace, w.flags);
-    p.tickets = at<uint32_t>(workspace, w.dec_tickets);
+    p.rec_range = at<int2>(workspace, w.rec_range);
     p.partials = at<float>(workspace, w.partials);
     p.s = s;
-    return launch_status(launch_decode(p, tmK, tmV, (cudaStream_t)stream));
+    return launch_status(launch_decode(p, (cudaStream_t)stream));
 }
 
 int csa_decode(const csa_dims* d, const void* q, const void* k_cache, const void* v_cache,

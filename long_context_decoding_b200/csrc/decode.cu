@@ -21,13 +21,16 @@
 // every SM, so ragged lengths and budgets stay balanced.
 //
 // Per CTA: the page ids of its slice are resolved once into shared memory;
-// a producer warp streams each page's K and V tile (16 tokens x D, bf16) with
-// 2-D TMA tensor copies, 64 channels (128 bytes) per box, 128-byte swizzle,
-// into a ring of stages tracked by mbarriers; four consumer warps take pages
-// round-robin.  Per page a warp computes S^T = K Q^T (16 tokens x 8 heads)
-// with mma.sync m16n8k16 (K fragments by ldmatrix, Q^T fragments resident
-// in registers), masks it, runs the fp32 online softmax in the exp2 domain,
-// turns P into the B operand with movmatrix, and accumulates
+// every warp then streams its own pages (round-robin over the slice) with
+// 16-byte cp.async copies into a private double buffer, laid out with the
+// 128-byte XOR swizzle (16-byte chunk c of token row r at c ^ (r & 7)), so
+// ldmatrix reads it without bank conflicts; slots past the end of the
+// sequence are zero-filled by the copy itself.  (Per-page TMA copies were
+// measured slower here: their issue cost, paid serially by one thread, caps
+// a CTA's request rate.)  Per page a warp computes S^T = K Q^T (16 tokens x
+// 8 heads) with mma.sync m16n8k16 (K fragments by ldmatrix, Q^T fragments
+// resident in registers), masks it, runs the fp32 online softmax in the exp2
+// domain, turns P into the B operand with movmatrix, and accumulates
 // O^T += V^T P^T with ldmatrix.trans fragments of V.  At the end of a unit
 // the warps merge through shared memory; a unit split over several CTAs
 // leaves one partial record (m, l, o) per CTA in the workspace, and the CTA
@@ -40,29 +43,39 @@ namespace {
 
 template <int D, int NB>
 struct DecCfg {
-    static constexpr int kConsumers = 4;
-    static constexpr int kThreads = 32 * (kConsumers + 1);
-    static constexpr int kBoxes = D / 64;               // 64-channel TMA boxes per K (or V) page
-    static constexpr int kHalf = kBoxes * 2048;         // bytes of one page's K (or V) tile
-    static constexpr int kStageBytes = 2 * kHalf;
-    static constexpr int kStages = D == 256 ? 4 : (D == 128 ? 8 : 16);
-    // a stage's previous use must belong to the same consumer warp, so that a
-    // parity wait can never be two phases ahead of the barrier
-    static_assert(kStages % kConsumers == 0, "stages must be a multiple of consumers");
+    static constexpr int kWarps = D == 256 ? 8 : 4;
+    static constexpr int kThreads = 32 * kWarps;
+    static constexpr int kBufs = D == 256 ? 1 : 2;      // page buffers per warp
+    static constexpr int kHalf = 32 * D;                // bytes of one page's K (or V) tile
+    static constexpr int kPageBytes = 2 * kHalf;
     static constexpr int kHeads = 8 * NB;               // query heads per CTA (padded)
     static constexpr int kMB = D / 16;                  // 16-channel blocks
-    static constexpr size_t kOw = (size_t)kConsumers * kHeads * D * 4;
-    static constexpr size_t kMl = (size_t)2 * kConsumers * kHeads * 4;
+    static constexpr size_t kStageArea = (size_t)kWarps * kBufs * kPageBytes;
+    static constexpr size_t kOw = (size_t)kWarps * kHeads * D * 4;   // aliases the stage area
+    static_assert(kOw <= kStageArea, "the merge buffer lives in the stage area");
+    static constexpr size_t kMl = (size_t)2 * kWarps * kHeads * 4;
     static constexpr size_t kItems = (size_t)kDecodeItemCap * 8;
     static __host__ __device__ size_t smem_bytes(int units) {
-        return 1024 /* alignment slack */ + (size_t)kStages * kStageBytes + kOw + kMl + kItems +
-               unit_bytes(units) + 16 * (size_t)kStages;
+        return 1024 /* alignment slack */ + kStageArea + kMl + kItems + unit_bytes(units);
     }
     // uoff [units + 1] | uinfo [units] (int2: seq_len, n_sel | n_blo << 30 | n_bhi << 31)
     static __host__ __device__ size_t unit_bytes(int units) {
         return (((size_t)(units + 1) * 4 + 15) & ~(size_t)15) + (size_t)units * 8;
     }
 };
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // What one unit reads, as counts of the five page groups of its work list.
 struct UnitPlan {
@@ -76,7 +89,11 @@ __device__ UnitPlan make_plan(const DecodeParams& p, int u) {
     UnitPlan q;
     q.b = u / p.s.Hkv;
     q.g = u % p.s.Hkv;
+    // first round of loads together: length, selection count, first entry
     int L = p.seq_lens[q.b];
+    const int32_t* sel_u = p.dense ? nullptr : p.sel + (size_t)u * p.s.max_sel;
+    int ns = p.dense ? 0 : p.n_sel[u];
+    const int first_raw = p.dense ? -1 : sel_u[0];
     if (L < 0 || L > p.s.MP * kPage) {
         latch_flag(p.flags, CSA_DEVFLAG_BAD_SEQ_LEN);
         L = 0;
@@ -97,16 +114,15 @@ __device__ UnitPlan make_plan(const DecodeParams& p, int u) {
     }
     q.n_pre = sg.c_lo;
     q.n_win = sg.np - sg.c_hi;
-    int ns = p.n_sel[u];
     const int cap = p.s.max_sel < sg.c_hi - sg.c_lo ? p.s.max_sel : sg.c_hi - sg.c_lo;
     if (ns < 0 || ns > cap) {
         latch_flag(p.flags, CSA_DEVFLAG_BAD_SELECTION);
         ns = ns < 0 ? 0 : cap;
     }
     q.n_sel = ns;
-    q.sel = p.sel + (size_t)u * p.s.max_sel;
-    const int first = ns > 0 ? q.sel[0] : -1;
-    const int last = ns > 0 ? q.sel[ns - 1] : -1;
+    q.sel = sel_u;
+    const int first = ns > 0 ? first_raw : -1;
+    const int last = ns > 0 ? sel_u[ns - 1] : -1;
     const bool lo_partial = (sg.Pe % kPage) != 0;
     const bool hi_partial = sg.We > 0 && ((L - sg.We) % kPage) != 0;
     q.n_blo = (lo_partial && first != sg.c_lo) ? 1 : 0;
@@ -181,115 +197,136 @@ __device__ __forceinline__ int cta_of(long long x, long long T, int n) {
     return (int)(i < n - 1 ? i : n - 1);
 }
 
-__device__ __forceinline__ void consumer_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(4 * 32) : "memory");
+// Partial record of one (CTA, unit): o[G][D] relative to the CTA's own max,
+// then m[G] (max, exp2 domain) and l[G] (sum); the stride keeps o 16-byte
+// aligned.
+__host__ __device__ __forceinline__ size_t record_stride(int G, int D) {
+    return ((size_t)G * D + 2 * G + 3) & ~(size_t)3;
 }
 
-// The CTA holding a unit's last ticket merges the unit's partial records
-// (o relative to its own max m, with m and l) written by CTAs
-// first .. last:  M = max_r m_r,  w_r = 2^(m_r - M),  out = sum_r w_r o_r /
-// sum_r w_r l_r.  Records are read through L2 in chunks: the weights of a
-// chunk go to shared memory first, then every thread sums its (head, channel)
-// elements with independent loads.
+// Combine kernel: merges the partial records of every unit split over
+// several decode CTAs, written by CTAs first .. last (rec_range):
+//   M = max_r m_r,  out = sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r.
+// A CTA covers 64 float4 columns of one unit's [G][D] output; its 256 threads
+// split the records four ways (online max-rescaled sums, merged with
+// shuffles), so no thread walks all the records.
+constexpr int kCombineCols = 64;
+
 template <int D>
-__device__ void merge_records(const DecodeParams& p, int b, int g, int u, int first, int last,
-                              size_t rec_stride, float* wsm, float* Msm, float* Lsm, int ctid) {
+__global__ void __launch_bounds__(256) combine_kernel(DecodeParams p) {
+    pdl_wait();                 // the records belong to the decode kernel
+    pdl_launch_dependents();
+    const int u = blockIdx.y;
+    const int2 rr = p.rec_range[u];
+    if (rr.y < rr.x) return;   // unit handled by a single CTA (or empty)
     const int G = p.s.G, Hq = p.s.Hq;
-    const int nrec = last - first + 1;
-    const float* base = p.partials + ((size_t)first + u) * rec_stride;
-    // M and L per head: one warp per head, lanes over records
-    const int warp = ctid >> 5, lane = ctid & 31;
-    for (int h = warp; h < G; h += 4) {
-        float m = -INFINITY;
-        for (int r = lane; r < nrec; r += 32)
-            m = fmaxf(m, __ldcg(base + (size_t)r * rec_stride + (size_t)h * (D + 2) + D));
+    const int cols = G * D / 4;
+    const int c = blockIdx.x * kCombineCols + (threadIdx.x & (kCombineCols - 1));
+    const int grp = threadIdx.x / kCombineCols;      // 0..3: record subset
+    if (blockIdx.x * kCombineCols >= cols) return;
+    const int cc = c < cols ? c : cols - 1;
+    const int h = (4 * cc) / D;
+    const size_t rs = record_stride(G, D);
+    const float* base = p.partials + ((size_t)rr.x + u) * rs;
+    const int nrec = rr.y - rr.x + 1;
+    float m = -INFINITY, l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r0 = grp; r0 < nrec; r0 += 4 * 4) {
+        float mr[4], lr[4];
+        float4 v[4];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float l = 0.f;
-        for (int r = lane; r < nrec; r += 32) {
-            const float* rc = base + (size_t)r * rec_stride + (size_t)h * (D + 2);
-            const float mr = __ldcg(rc + D);
-            l += mr == -INFINITY ? 0.f : __ldcg(rc + D + 1) * ex2(mr - m);
+        for (int k = 0; k < 4; ++k) {
+            const int r = r0 + 4 * k;
+            const float* rc = base + (size_t)(r < nrec ? r : 0) * rs;
+            mr[k] = r < nrec ? __ldcg(rc + (size_t)G * D + h) : -INFINITY;
+            lr[k] = __ldcg(rc + (size_t)G * D + G + h);
+            v[k] = __ldcg(reinterpret_cast<const float4*>(rc) + cc);
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (lane == 0) {
-            Msm[h] = m;
-            Lsm[h] = l;
+        for (int k = 0; k < 4; ++k) {
+            if (mr[k] == -INFINITY) continue;
+            const float mn = fmaxf(m, mr[k]);
+            const float a = m == -INFINITY ? 0.f : ex2(m - mn), w = ex2(mr[k] - mn);
+            acc.x = acc.x * a + v[k].x * w;
+            acc.y = acc.y * a + v[k].y * w;
+            acc.z = acc.z * a + v[k].z * w;
+            acc.w = acc.w * a + v[k].w * w;
+            l = l * a + lr[k] * w;
+            m = mn;
         }
     }
-    consumer_sync();
-    constexpr int kPer = 8;                       // elements per thread and pass
-    const int total = G * D;
-    const int chunk = (4 * 8 * D) / G;            // records whose weights fit in wsm
-    for (int e0 = 0; e0 < total; e0 += 128 * kPer) {
-        float acc[kPer];
+    // merge the four record groups (threads t, t+64, t+128, t+192)
+    __shared__ float sm[4][kCombineCols][6];
+    const int col = threadIdx.x & (kCombineCols - 1);
+    sm[grp][col][0] = m;
+    sm[grp][col][1] = l;
+    sm[grp][col][2] = acc.x;
+    sm[grp][col][3] = acc.y;
+    sm[grp][col][4] = acc.z;
+    sm[grp][col][5] = acc.w;
+    __syncthreads();
+    if (grp != 0 || c >= cols) return;
+    float M = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
-        for (int r0 = 0; r0 < nrec; r0 += chunk) {
-            const int rn = nrec - r0 < chunk ? nrec - r0 : chunk;
-            for (int i = ctid; i < rn * G; i += 128) {
-                const int r = r0 + i / G, h = i % G;
-                const float mr = __ldcg(base + (size_t)r * rec_stride + (size_t)h * (D + 2) + D);
-                wsm[i] = mr == -INFINITY ? 0.f : ex2(mr - Msm[h]);
-            }
-            consumer_sync();
-            for (int r = 0; r < rn; ++r) {
-                const float* rc = base + (size_t)(r0 + r) * rec_stride;
+    for (int g2 = 0; g2 < 4; ++g2) M = fmaxf(M, sm[g2][col][0]);
+    float L = 0.f, o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
 #pragma unroll
-                for (int j = 0; j < kPer; ++j) {
-                    const int idx = e0 + j * 128 + ctid;
-                    if (idx < total) {
-                        const int h = idx / D, c = idx % D;
-                        acc[j] += __ldcg(rc + (size_t)h * (D + 2) + c) * wsm[r * G + h];
-                    }
-                }
-            }
-            consumer_sync();
-        }
+    for (int g2 = 0; g2 < 4; ++g2) {
+        const float mg = sm[g2][col][0];
+        const float f = mg == -INFINITY ? 0.f : ex2(mg - M);
+        L += sm[g2][col][1] * f;
+        o0 += sm[g2][col][2] * f;
+        o1 += sm[g2][col][3] * f;
+        o2 += sm[g2][col][4] * f;
+        o3 += sm[g2][col][5] * f;
+    }
+    const int b = u / p.s.Hkv, g = u % p.s.Hkv;
+    const int ch = (4 * c) % D;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const size_t oi = (size_t)b * Hq + (size_t)g * G + h;
+    uint2 pk;
+    pk.x = pack_bf16x2(o0 * inv, o1 * inv);
+    pk.y = pack_bf16x2(o2 * inv, o3 * inv);
+    *reinterpret_cast<uint2*>(p.out + oi * D + ch) = pk;
+    if (ch == 0 && p.lse) p.lse[oi] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+// Issues the cp.async copies of one page's K and V tiles (16 tokens x D) into
+// a swizzled buffer; token rows >= rows_valid are zero-filled.
+template <int D>
+__device__ __forceinline__ void load_page(uint32_t buf, const uint16_t* kt, const uint16_t* vt,
+                                          int rows_valid, int lane) {
+    constexpr int kChunksPerRow = D / 8;
+    constexpr int kChunks = 16 * kChunksPerRow;
 #pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int idx = e0 + j * 128 + ctid;
-            if (idx < total) {
-                const int h = idx / D, c = idx % D;
-                const float l = Lsm[h];
-                const size_t oi = (size_t)b * Hq + (size_t)g * G + h;
-                p.out[oi * D + c] =
-                    __bfloat16_as_ushort(__float2bfloat16_rn(l > 0.f ? acc[j] / l : 0.f));
-                if (c == 0 && p.lse)
-                    p.lse[oi] = l > 0.f ? (Msm[h] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-            }
-        }
+    for (int i = 0; i < kChunks / 32; ++i) {
+        const int idx = i * 32 + lane;
+        const int r = idx / kChunksPerRow, c16 = idx % kChunksPerRow;
+        const uint32_t off = (c16 >> 3) * 2048 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+        const uint32_t n = r < rows_valid ? 16u : 0u;
+        cp_async_16(buf + off, kt + (size_t)r * D + c16 * 8, n);
+        cp_async_16(buf + 32 * D + off, vt + (size_t)r * D + c16 * 8, n);
     }
 }
 
 template <int D, int NB>
 __global__ void __launch_bounds__(DecCfg<D, NB>::kThreads)
-decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-              DecodeParams p) {
+decode_kernel(DecodeParams p) {
     using C = DecCfg<D, NB>;
-    static_assert(C::kConsumers == 4, "consumer_sync counts 4 warps");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // swizzled TMA destinations need 1024-byte alignment in the shared window
+    // swizzled page buffers need 1024-byte alignment in the shared window
     uint8_t* stages = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    float* Ow = reinterpret_cast<float*>(stages + (size_t)C::kStages * C::kStageBytes);
-    float* ms = Ow + C::kConsumers * C::kHeads * D;
-    float* ls = ms + C::kConsumers * C::kHeads;
-    int2* items = reinterpret_cast<int2*>(ls + C::kConsumers * C::kHeads);
+    float* Ow = reinterpret_cast<float*>(stages);      // reused after the page loop
+    float* ms = reinterpret_cast<float*>(stages + C::kStageArea);
+    float* ls = ms + C::kWarps * C::kHeads;
+    int2* items = reinterpret_cast<int2*>(ls + C::kWarps * C::kHeads);
     int* uoff = reinterpret_cast<int*>(items + kDecodeItemCap);
     const int units = p.s.B * p.s.Hkv;
     int2* uinfo = reinterpret_cast<int2*>(reinterpret_cast<uint8_t*>(uoff) +
                                           (((size_t)(units + 1) * 4 + 15) & ~(size_t)15));
-    uint64_t* full = reinterpret_cast<uint64_t*>(uinfo + units);
-    uint64_t* empty = full + C::kStages;
-    __shared__ int s_abort, s_last, s_issued;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Hkv = p.s.Hkv, G = p.s.G, Hq = p.s.Hq;
-    if (tid == 0) {
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
-    }
     // the selection, the appended tokens and the previous users of the
     // workspace belong to earlier kernels
     pdl_wait();
@@ -300,10 +337,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         const UnitPlan q = make_plan(p, u);
         uoff[u] = q.total();
         uinfo[u] = make_int2(q.L, q.n_sel | (q.n_blo << 30) | (q.n_bhi << 31));
-    }
-    if (tid == 0) {
-        s_abort = 0;
-        s_issued = 0;
     }
     __syncthreads();
     if (warp == 0) {
@@ -327,7 +360,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     // partition over at most T CTAs so that every participating CTA owns at
     // least one item: the merge counts every CTA between a unit's first and
     // last one
-    const int n_cta = (int)(T < (long long)gridDim.x ? (T > 0 ? T : 1) : gridDim.x);
+    // at least kMinItems pages per CTA: fewer partial records per unit to
+    // merge when the attended set is small
+    constexpr long long kMinItems = 4 * C::kWarps;
+    long long want = (T + kMinItems - 1) / kMinItems;
+    if (want < 1) want = 1;
+    const int n_cta = (int)(want < (long long)gridDim.x ? want : gridDim.x);
     const long long s = blockIdx.x < (unsigned)n_cta ? T * blockIdx.x / n_cta : T;
     const long long e = blockIdx.x < (unsigned)n_cta ? T * (blockIdx.x + 1) / n_cta : T;
 
@@ -335,6 +373,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     if (blockIdx.x == 0) {
         for (int u = 0; u < units; ++u) {
             if (uoff[u + 1] != uoff[u]) continue;
+            if (tid == 0) p.rec_range[u] = make_int2(0, -1);
             const int b = u / Hkv, g = u % Hkv;
             for (int i = tid; i < G * D; i += C::kThreads) {
                 const int h = i / D, c = i % D;
@@ -363,289 +402,230 @@ decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         }
         items[x - s] = make_int2(phys, page * 2 + (whole ? 1 : 0));
     }
-    if (tid == 0) {
-        for (int i = 0; i < C::kStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-        }
-        fence_barrier_init();
-    }
     __syncthreads();
 
     const int u_first = find_unit(uoff, units, s);
     const int u_last = find_unit(uoff, units, e - 1);
+    const int gq = lane >> 2, tq = lane & 3;
+    const int mi = lane >> 3, ri = lane & 7;
+    // per-lane ldmatrix geometry (chunk c of row r sits at c ^ (r & 7))
+    const int k_tok = ri + ((mi & 1) << 3), k_half = mi >> 1;
+    const int v_tok = ri + ((mi >> 1) << 3), v_half = mi & 1;
+    const float sl2 = p.scale_log2;
+    const uint32_t wbuf = smem_u32(stages) + (uint32_t)(warp * C::kBufs * C::kPageBytes);
 
-    if (warp == C::kConsumers) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-            int u = u_first;
-            for (long long x = s; x < e; ++x) {
-                while (x >= uoff[u + 1]) ++u;
-                const int i = (int)(x - s);
-                const int st = i % C::kStages, r = i / C::kStages;
-                if (r > 0 && !mbar_wait(&empty[st], (r - 1) & 1)) {
-                    latch_flag(p.flags, CSA_DEVFLAG_TIMEOUT);
-                    s_abort = 1;
-                }
-                if (*(volatile int*)&s_abort) break;
-                const int2 it = items[i];
-                if (it.x >= 0) {
-                    const int row = (it.x * Hkv + (u % Hkv)) * kPage;
-                    uint8_t* dst = stages + (size_t)st * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+    for (int u = u_first; u <= u_last; ++u) {
+        const long long a = s > uoff[u] ? s : uoff[u];
+        const long long bnd = e < uoff[u + 1] ? e : uoff[u + 1];
+        if (a >= bnd) continue;
+        const int b = u / Hkv, g = u % Hkv;
+        const int L = uinfo[u].x;
+        const SeqGeom sg = seq_geom(L, p.prefix, p.window);
+        const int Pe = sg.Pe, Lw = L - sg.We;
+
+        // Q^T as the B operand: b0 = q[head][16kb + 2tq, +1], b1 = +8
+        uint32_t qf[C::kMB][NB][2];
 #pragma unroll
-                    for (int bx = 0; bx < C::kBoxes; ++bx) {
-                        tma_tile_g2s(dst + bx * 2048, &tmK, bx * 64, row, &full[st]);
-                        tma_tile_g2s(dst + C::kHalf + bx * 2048, &tmV, bx * 64, row, &full[st]);
-                    }
-                } else {
-                    mbar_arrive(&full[st]);
-                }
-                s_issued = i + 1;
+        for (int nb = 0; nb < NB; ++nb) {
+            const int head = nb * 8 + gq;
+            const uint32_t* qw = reinterpret_cast<const uint32_t*>(
+                p.q + ((size_t)b * Hq + (size_t)g * G + (head < G ? head : 0)) * D);
+#pragma unroll
+            for (int kb = 0; kb < C::kMB; ++kb) {
+                qf[kb][nb][0] = head < G ? __ldg(qw + 8 * kb + tq) : 0u;
+                qf[kb][nb][1] = head < G ? __ldg(qw + 8 * kb + 4 + tq) : 0u;
             }
         }
-    } else {
-        // ------------------------------------------------------------ consumers
-        const int gq = lane >> 2, tq = lane & 3;
-        const int mi = lane >> 3, ri = lane & 7;
-        // per-lane ldmatrix geometry (128-byte swizzle: chunk c of row r sits at c ^ (r & 7))
-        const int k_tok = ri + ((mi & 1) << 3), k_half = mi >> 1;
-        const int v_tok = ri + ((mi >> 1) << 3), v_half = mi & 1;
-        const float sl2 = p.scale_log2;
-
-        for (int u = u_first; u <= u_last; ++u) {
-            const long long a = s > uoff[u] ? s : uoff[u];
-            const long long bnd = e < uoff[u + 1] ? e : uoff[u + 1];
-            if (a >= bnd) continue;
-            const int b = u / Hkv, g = u % Hkv;
-            int L = p.seq_lens[b];
-            if (L < 0 || L > p.s.MP * kPage) L = 0;
-            const SeqGeom sg = seq_geom(L, p.prefix, p.window);
-            const int Pe = sg.Pe, Lw = L - sg.We;
-
-            // Q^T as the B operand: b0 = q[head][16kb + 2tq, +1], b1 = +8
-            uint32_t qf[C::kMB][NB][2];
+        float m[NB][2], l[NB][2], o[C::kMB][NB][4];
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const int head = nb * 8 + gq;
-                const uint32_t* qw = reinterpret_cast<const uint32_t*>(
-                    p.q + ((size_t)b * Hq + (size_t)g * G + (head < G ? head : 0)) * D);
+        for (int nb = 0; nb < NB; ++nb) {
+            m[nb][0] = m[nb][1] = -INFINITY;
+            l[nb][0] = l[nb][1] = 0.f;
+#pragma unroll
+            for (int mb = 0; mb < C::kMB; ++mb)
+                o[mb][nb][0] = o[mb][nb][1] = o[mb][nb][2] = o[mb][nb][3] = 0.f;
+        }
+
+        // this warp's items of the segment: a + warp, a + warp + kWarps, ...
+        auto issue = [&](long long x, int slot) {
+            const int2 it = items[x - s];
+            if (it.x >= 0) {
+                const int page = it.y >> 1;
+                const size_t tile = ((size_t)it.x * Hkv + g) * kPage * D;
+                const int rows = L - page * kPage < kPage ? L - page * kPage : kPage;
+                load_page<D>(wbuf + (uint32_t)(slot * C::kPageBytes), p.k_cache + tile,
+                             p.v_cache + tile, rows, lane);
+            }
+            cp_async_commit();
+        };
+        long long x = a + warp;
+        int slot = 0;
+        if (x < bnd) issue(x, 0);
+        for (; x < bnd; x += C::kWarps) {
+            const long long xn = x + C::kWarps;
+            if (C::kBufs == 2) {
+                if (xn < bnd) {
+                    issue(xn, slot ^ 1);
+                    cp_async_wait<1>();
+                } else {
+                    cp_async_wait<0>();
+                }
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncwarp();
+            const int2 it = items[x - s];
+            if (it.x >= 0) {
+                const int page = it.y >> 1;
+                const bool whole = it.y & 1;
+                const uint32_t kbase = wbuf + (uint32_t)(slot * C::kPageBytes);
+                const uint32_t vbase = kbase + C::kHalf;
+                // ---- S^T = K Q^T
+                float sacc[NB][4];
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb)
+                    sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
 #pragma unroll
                 for (int kb = 0; kb < C::kMB; ++kb) {
-                    qf[kb][nb][0] = head < G ? __ldg(qw + 8 * kb + tq) : 0u;
-                    qf[kb][nb][1] = head < G ? __ldg(qw + 8 * kb + 4 + tq) : 0u;
-                }
-            }
-            float m[NB][2], l[NB][2], o[C::kMB][NB][4];
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                m[nb][0] = m[nb][1] = -INFINITY;
-                l[nb][0] = l[nb][1] = 0.f;
-#pragma unroll
-                for (int mb = 0; mb < C::kMB; ++mb)
-                    o[mb][nb][0] = o[mb][nb][1] = o[mb][nb][2] = o[mb][nb][3] = 0.f;
-            }
-
-            for (long long x = a; x < bnd; ++x) {
-                const int i = (int)(x - s);
-                if (i % C::kConsumers != warp) continue;
-                const int st = i % C::kStages, r = i / C::kStages;
-                if (!*(volatile int*)&s_abort && !mbar_wait(&full[st], r & 1)) {
-                    if (lane == 0) latch_flag(p.flags, CSA_DEVFLAG_TIMEOUT);
-                    s_abort = 1;
-                }
-                const int2 it = items[i];
-                bool wrote = false;
-                if (!*(volatile int*)&s_abort && it.x >= 0) {
-                    const int page = it.y >> 1;
-                    const bool whole = it.y & 1;
-                    const uint32_t kbase = smem_u32(stages + (size_t)st * C::kStageBytes);
-                    const uint32_t vbase = kbase + C::kHalf;
-                    // ---- S^T = K Q^T
-                    float sacc[NB][4];
+                    const int chunk = 2 * kb + k_half;
+                    const uint32_t addr = kbase + (chunk >> 3) * 2048 + k_tok * 128 +
+                                          (((chunk & 7) ^ ri) << 4);
+                    uint32_t af[4];
+                    ldsm_x4(af, addr);
 #pragma unroll
                     for (int nb = 0; nb < NB; ++nb)
-                        sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
+                        mma_bf16_16816(sacc[nb], af, qf[kb][nb][0], qf[kb][nb][1]);
+                }
+                // ---- mask and online softmax (exp2 domain)
+                const int t0 = page * kPage + gq, t1 = t0 + 8;
+                const bool in0 = t0 < L && (whole || t0 < Pe || t0 >= Lw);
+                const bool in1 = t1 < L && (whole || t1 < Pe || t1 >= Lw);
+                uint32_t pb[NB][2];
 #pragma unroll
-                    for (int kb = 0; kb < C::kMB; ++kb) {
-                        const int chunk = 2 * kb + k_half;
-                        const uint32_t addr = kbase + (chunk >> 3) * 2048 + k_tok * 128 +
-                                              (((chunk & 7) ^ ri) << 4);
-                        uint32_t af[4];
-                        ldsm_x4(af, addr);
+                for (int nb = 0; nb < NB; ++nb) {
+                    const float s00 = in0 ? sacc[nb][0] * sl2 : -INFINITY;
+                    const float s01 = in0 ? sacc[nb][1] * sl2 : -INFINITY;
+                    const float s10 = in1 ? sacc[nb][2] * sl2 : -INFINITY;
+                    const float s11 = in1 ? sacc[nb][3] * sl2 : -INFINITY;
+                    float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
 #pragma unroll
-                        for (int nb = 0; nb < NB; ++nb)
-                            mma_bf16_16816(sacc[nb], af, qf[kb][nb][0], qf[kb][nb][1]);
+                    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
                     }
-                    // ---- mask and online softmax (exp2 domain)
-                    const int t0 = page * kPage + gq, t1 = t0 + 8;
-                    const bool in0 = t0 < L && (whole || t0 < Pe || t0 >= Lw);
-                    const bool in1 = t1 < L && (whole || t1 < Pe || t1 >= Lw);
-                    uint32_t pb[NB][2];
-#pragma unroll
-                    for (int nb = 0; nb < NB; ++nb) {
-                        const float s00 = in0 ? sacc[nb][0] * sl2 : -INFINITY;
-                        const float s01 = in0 ? sacc[nb][1] * sl2 : -INFINITY;
-                        const float s10 = in1 ? sacc[nb][2] * sl2 : -INFINITY;
-                        const float s11 = in1 ? sacc[nb][3] * sl2 : -INFINITY;
-                        float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
-#pragma unroll
-                        for (int o2 = 4; o2 < 32; o2 <<= 1) {
-                            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
-                            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
-                        }
-                        const float mn0 = fmaxf(m[nb][0], mx0), mn1 = fmaxf(m[nb][1], mx1);
-                        const float base0 = mn0 == -INFINITY ? 0.f : mn0;
-                        const float base1 = mn1 == -INFINITY ? 0.f : mn1;
-                        const float al0 = ex2(m[nb][0] - base0), al1 = ex2(m[nb][1] - base1);
-                        const uint32_t P0 = pack_bf16x2(ex2(s00 - base0), ex2(s01 - base1));
-                        const uint32_t P1 = pack_bf16x2(ex2(s10 - base0), ex2(s11 - base1));
-                        l[nb][0] = l[nb][0] * al0 + bf16_lo(P0) + bf16_lo(P1);
-                        l[nb][1] = l[nb][1] * al1 + bf16_hi(P0) + bf16_hi(P1);
-                        m[nb][0] = mn0;
-                        m[nb][1] = mn1;
-#pragma unroll
-                        for (int mb = 0; mb < C::kMB; ++mb) {
-                            o[mb][nb][0] *= al0;
-                            o[mb][nb][1] *= al1;
-                            o[mb][nb][2] *= al0;
-                            o[mb][nb][3] *= al1;
-                        }
-                        pb[nb][0] = movmatrix_trans(P0);
-                        pb[nb][1] = movmatrix_trans(P1);
-                    }
-                    // ---- slots past the end of the sequence may hold anything:
-                    // zero those V rows so that P = 0 cannot meet a NaN
-                    if (page == sg.np - 1 && (L & (kPage - 1))) {
-                        const int r0 = L & (kPage - 1);
-                        for (int c = lane; c < C::kBoxes * 128; c += 32) {
-                            const int row = (c >> 3) & 15;
-                            if (row >= r0) {
-                                const uint32_t za = vbase + (c >> 7) * 2048 + row * 128 + (c & 7) * 16;
-                                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(za),
-                                             "r"(0u)
-                                             : "memory");
-                            }
-                        }
-                        __syncwarp();
-                        wrote = true;
-                    }
-                    // ---- O^T += V^T P^T
+                    const float mn0 = fmaxf(m[nb][0], mx0), mn1 = fmaxf(m[nb][1], mx1);
+                    const float base0 = mn0 == -INFINITY ? 0.f : mn0;
+                    const float base1 = mn1 == -INFINITY ? 0.f : mn1;
+                    const float al0 = ex2(m[nb][0] - base0), al1 = ex2(m[nb][1] - base1);
+                    const uint32_t P0 = pack_bf16x2(ex2(s00 - base0), ex2(s01 - base1));
+                    const uint32_t P1 = pack_bf16x2(ex2(s10 - base0), ex2(s11 - base1));
+                    l[nb][0] = l[nb][0] * al0 + bf16_lo(P0) + bf16_lo(P1);
+                    l[nb][1] = l[nb][1] * al1 + bf16_hi(P0) + bf16_hi(P1);
+                    m[nb][0] = mn0;
+                    m[nb][1] = mn1;
 #pragma unroll
                     for (int mb = 0; mb < C::kMB; ++mb) {
-                        const int chunk = 2 * mb + v_half;
-                        const uint32_t addr = vbase + (chunk >> 3) * 2048 + v_tok * 128 +
-                                              (((chunk & 7) ^ ri) << 4);
-                        uint32_t af[4];
-                        ldsm_x4_trans(af, addr);
-#pragma unroll
-                        for (int nb = 0; nb < NB; ++nb)
-                            mma_bf16_16816(o[mb][nb], af, pb[nb][0], pb[nb][1]);
+                        o[mb][nb][0] *= al0;
+                        o[mb][nb][1] *= al1;
+                        o[mb][nb][2] *= al0;
+                        o[mb][nb][3] *= al1;
                     }
+                    pb[nb][0] = movmatrix_trans(P0);
+                    pb[nb][1] = movmatrix_trans(P1);
                 }
-                __syncwarp();
-                if (lane == 0) {
-                    if (wrote) fence_proxy_async_smem();
-                    mbar_arrive(&empty[st]);
-                }
-            }
-
-            // ---- merge the four warps of this CTA
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float v = l[nb][hh];
-                    v += __shfl_xor_sync(0xffffffffu, v, 4);
-                    v += __shfl_xor_sync(0xffffffffu, v, 8);
-                    v += __shfl_xor_sync(0xffffffffu, v, 16);
-                    l[nb][hh] = v;
-                }
-                if (gq == 0) {
-                    ms[warp * C::kHeads + nb * 8 + 2 * tq] = m[nb][0];
-                    ms[warp * C::kHeads + nb * 8 + 2 * tq + 1] = m[nb][1];
-                    ls[warp * C::kHeads + nb * 8 + 2 * tq] = l[nb][0];
-                    ls[warp * C::kHeads + nb * 8 + 2 * tq + 1] = l[nb][1];
-                }
+                // ---- O^T += V^T P^T
 #pragma unroll
                 for (int mb = 0; mb < C::kMB; ++mb) {
-                    float* ow = Ow + (size_t)warp * C::kHeads * D;
-                    const int h0 = nb * 8 + 2 * tq, c0 = mb * 16 + gq;
-                    ow[(size_t)h0 * D + c0] = o[mb][nb][0];
-                    ow[(size_t)(h0 + 1) * D + c0] = o[mb][nb][1];
-                    ow[(size_t)h0 * D + c0 + 8] = o[mb][nb][2];
-                    ow[(size_t)(h0 + 1) * D + c0 + 8] = o[mb][nb][3];
+                    const int chunk = 2 * mb + v_half;
+                    const uint32_t addr = vbase + (chunk >> 3) * 2048 + v_tok * 128 +
+                                          (((chunk & 7) ^ ri) << 4);
+                    uint32_t af[4];
+                    ldsm_x4_trans(af, addr);
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+                        mma_bf16_16816(o[mb][nb], af, pb[nb][0], pb[nb][1]);
                 }
             }
-            consumer_sync();
+            __syncwarp();                 // the buffer is refilled next
+            if (C::kBufs == 1) {
+                if (xn < bnd) issue(xn, 0);
+            } else {
+                slot ^= 1;
+            }
+        }
 
-            const int first_cta = cta_of(uoff[u], T, n_cta);
-            const int last_cta = cta_of(uoff[u + 1] - 1, T, n_cta);
-            const bool alone = first_cta == last_cta;
-            const int ctid = tid;                      // 0 .. 127
-            const size_t rec_stride = (size_t)G * (D + 2);
-            float* rec = p.partials + ((size_t)blockIdx.x + u) * rec_stride;
-            for (int idx = ctid; idx < G * D; idx += 128) {
-                const int h = idx / D, c = idx % D;
-                float M = -INFINITY;
+        // ---- merge the warps of this CTA (Ow aliases the page buffers)
+        __syncthreads();
 #pragma unroll
-                for (int w = 0; w < C::kConsumers; ++w) M = fmaxf(M, ms[w * C::kHeads + h]);
-                float acc = 0.f, lsum = 0.f;
+        for (int nb = 0; nb < NB; ++nb) {
 #pragma unroll
-                for (int w = 0; w < C::kConsumers; ++w) {
-                    const float mw = ms[w * C::kHeads + h];
-                    const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
-                    acc += Ow[((size_t)w * C::kHeads + h) * D + c] * f;
-                    lsum += ls[w * C::kHeads + h] * f;
-                }
-                const size_t oi = ((size_t)b * Hq + (size_t)g * G + h);
-                if (alone) {
-                    const float val = lsum > 0.f ? acc / lsum : 0.f;
-                    p.out[oi * D + c] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
-                    if (c == 0 && p.lse)
-                        p.lse[oi] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f
-                                               : -INFINITY;
-                } else {
-                    rec[(size_t)h * (D + 2) + c] = acc;
-                    if (c == 0) {
-                        rec[(size_t)h * (D + 2) + D] = M;
-                        rec[(size_t)h * (D + 2) + D + 1] = lsum;
-                    }
+            for (int hh = 0; hh < 2; ++hh) {
+                float v = l[nb][hh];
+                v += __shfl_xor_sync(0xffffffffu, v, 4);
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                l[nb][hh] = v;
+            }
+            if (gq == 0) {
+                ms[warp * C::kHeads + nb * 8 + 2 * tq] = m[nb][0];
+                ms[warp * C::kHeads + nb * 8 + 2 * tq + 1] = m[nb][1];
+                ls[warp * C::kHeads + nb * 8 + 2 * tq] = l[nb][0];
+                ls[warp * C::kHeads + nb * 8 + 2 * tq + 1] = l[nb][1];
+            }
+#pragma unroll
+            for (int mb = 0; mb < C::kMB; ++mb) {
+                float* ow = Ow + (size_t)warp * C::kHeads * D;
+                const int h0 = nb * 8 + 2 * tq, c0 = mb * 16 + gq;
+                ow[(size_t)h0 * D + c0] = o[mb][nb][0];
+                ow[(size_t)(h0 + 1) * D + c0] = o[mb][nb][1];
+                ow[(size_t)h0 * D + c0 + 8] = o[mb][nb][2];
+                ow[(size_t)(h0 + 1) * D + c0 + 8] = o[mb][nb][3];
+            }
+        }
+        __syncthreads();
+
+        const int first_cta = cta_of(uoff[u], T, n_cta);
+        const int last_cta = cta_of(uoff[u + 1] - 1, T, n_cta);
+        const bool alone = first_cta == last_cta;
+        if (alone && tid == 0) p.rec_range[u] = make_int2(0, -1);   // nothing to combine
+        const size_t rs = record_stride(G, D);
+        float* rec = p.partials + ((size_t)blockIdx.x + u) * rs;
+        for (int idx = tid; idx < G * D; idx += C::kThreads) {
+            const int h = idx / D, c = idx % D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < C::kWarps; ++w) M = fmaxf(M, ms[w * C::kHeads + h]);
+            float acc = 0.f, lsum = 0.f;
+#pragma unroll
+            for (int w = 0; w < C::kWarps; ++w) {
+                const float mw = ms[w * C::kHeads + h];
+                const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
+                acc += Ow[((size_t)w * C::kHeads + h) * D + c] * f;
+                lsum += ls[w * C::kHeads + h] * f;
+            }
+            const size_t oi = ((size_t)b * Hq + (size_t)g * G + h);
+            if (alone) {
+                const float val = lsum > 0.f ? acc / lsum : 0.f;
+                p.out[oi * D + c] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+                if (c == 0 && p.lse)
+                    p.lse[oi] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f
+                                           : -INFINITY;
+            } else {
+                rec[(size_t)h * D + c] = acc;
+                if (c == 0) {
+                    rec[(size_t)G * D + h] = M;
+                    rec[(size_t)G * D + G + h] = lsum;
                 }
             }
-            if (!alone) {
-                __threadfence();
-                consumer_sync();
-                if (ctid == 0) {
-                    const unsigned prev = atomicAdd(&p.tickets[u], 1u);
-                    s_last = prev == (unsigned)(last_cta - first_cta);
-                }
-                consumer_sync();
-                if (s_last) {
-                    __threadfence();
-                    merge_records<D>(p, b, g, u, first_cta, last_cta, rec_stride, Ow, ms, ls,
-                                     ctid);
-                    if (ctid == 0) atomicExch(&p.tickets[u], 0u);
-                }
-            }
-            consumer_sync();   // Ow / ms / ls are reused by the next unit
         }
-    }
-    __syncthreads();
-    if (tid == 0 && s_abort) {    // bounded drain of copies still in flight
-        const int n = s_issued;
-        for (int st = 0; st < C::kStages && st < n; ++st) {
-            const int last = st + ((n - 1 - st) / C::kStages) * C::kStages;
-            mbar_wait(&full[st], (last / C::kStages) & 1);
-        }
+        if (!alone && blockIdx.x == first_cta && tid == 0)
+            p.rec_range[u] = make_int2(first_cta, last_cta);   // read by the combine kernel
+        __syncthreads();   // Ow / ms / ls and the page buffers are reused by the next unit
     }
 }
 
 template <int D, int NB>
-cudaError_t launch_decode_t(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                            cudaStream_t st) {
+cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t st) {
     using C = DecCfg<D, NB>;
     auto kern = decode_kernel<D, NB>;
     const int units = p.s.B * p.s.Hkv;
@@ -660,18 +640,22 @@ cudaError_t launch_decode_t(const DecodeParams& p, const CUtensorMap& tmK, const
         attr_done[dev] = 1;
     }
     const int grid = decode_grid(p.s);
-    return launch_pdl(decode_kernel<D, NB>, dim3(grid), dim3(C::kThreads), smem, st, tmK, tmV, p);
+    cudaError_t e = launch_pdl(kern, dim3(grid), dim3(C::kThreads), smem, st, p);
+    if (e != cudaSuccess) return e;
+    const int col_blocks = (p.s.G * D / 4 + kCombineCols - 1) / kCombineCols;
+    return launch_pdl(combine_kernel<D>, dim3(col_blocks, units), dim3(256), 0, st, p);
 }
 
 }  // namespace
 
-// Resident CTAs of the decode kernel for this shape, times the SM count, and
-// at least enough CTAs that no slice exceeds the per-CTA item capacity.
+// Resident CTAs of the decode kernel for this shape (shared memory decides),
+// times the SM count, and at least enough CTAs that no slice exceeds the
+// per-CTA item capacity.
 template <int D, int NB>
 static int resident_per_sm(int units) {
     const size_t per_cta = DecCfg<D, NB>::smem_bytes(units) + 1024;   // + per-CTA reserve
     int n = (int)((size_t)(228 * 1024) / per_cta);
-    if (n > 2) n = 2;
+    if (n > 3) n = 3;
     return n < 1 ? 1 : n;
 }
 
@@ -693,16 +677,17 @@ int decode_grid(const Shape& s) {
     return (int)(grid < 1 ? 1 : grid);
 }
 
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                          cudaStream_t st) {
+size_t decode_record_floats(const Shape& s) { return record_stride(s.G, s.D); }
+
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st) {
     const int nb = p.s.G > 8 ? 2 : 1;
     switch (p.s.D * 10 + nb) {
-        case 641: return launch_decode_t<64, 1>(p, tmK, tmV, st);
-        case 642: return launch_decode_t<64, 2>(p, tmK, tmV, st);
-        case 1281: return launch_decode_t<128, 1>(p, tmK, tmV, st);
-        case 1282: return launch_decode_t<128, 2>(p, tmK, tmV, st);
-        case 2561: return launch_decode_t<256, 1>(p, tmK, tmV, st);
-        case 2562: return launch_decode_t<256, 2>(p, tmK, tmV, st);
+        case 641: return launch_decode_t<64, 1>(p, st);
+        case 642: return launch_decode_t<64, 2>(p, st);
+        case 1281: return launch_decode_t<128, 1>(p, st);
+        case 1282: return launch_decode_t<128, 2>(p, st);
+        case 2561: return launch_decode_t<256, 1>(p, st);
+        case 2562: return launch_decode_t<256, 2>(p, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -13,9 +13,9 @@ namespace csa {
 struct WsLayout {
     size_t flags;          // uint32 device flag word
     size_t score_tickets;  // uint32 [units]
-    size_t dec_tickets;    // uint32 [units]
+    size_t rec_range;      // int2 [units]
     size_t scores;         // fp32 [B][Hkv][max_pages]
-    size_t partials;       // fp32 [dec_slots][G][D + 2]
+    size_t partials;       // fp32 [dec_slots][decode_record_floats]
     size_t dec_slots;      // partial records available
     size_t total;
 };
@@ -61,6 +61,7 @@ struct SelectParams {
     int32_t* sel;
     int32_t* n_sel;
     uint32_t* flags;
+    int smem_keys;          // keys that fit in the dynamic shared memory (set by the launcher)
     Shape s;
 };
 cudaError_t launch_select(const SelectParams& p, cudaStream_t st);
@@ -68,6 +69,8 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t st);
 // ---------------------------------------------------------------- decode
 struct DecodeParams {
     const uint16_t* q;
+    const uint16_t* k_cache;
+    const uint16_t* v_cache;
     const int32_t* page_table;
     const int32_t* seq_lens;
     const int32_t* sel;     // nullable when dense
@@ -78,16 +81,16 @@ struct DecodeParams {
     uint16_t* out;
     float* lse;             // nullable
     uint32_t* flags;
-    uint32_t* tickets;      // [units]
-    float* partials;        // [dec_slots][G][D + 2]
+    int2* rec_range;        // [units]: CTAs whose partial records the combine merges
+    float* partials;        // [dec_slots][record]: o[G][D] | m[G] | l[G]
     Shape s;
 };
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                          cudaStream_t st);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st);
 
 // Grid sizes (shared by the workspace sizing and the launches).
 int device_sm_count();
 int decode_grid(const Shape& s);
+size_t decode_record_floats(const Shape& s);   // floats per split-K partial record
 WsLayout workspace_layout(const Shape& s);
 
 }  // namespace csa

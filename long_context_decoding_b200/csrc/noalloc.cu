@@ -7,7 +7,7 @@
 // for its KV cache at start-up and forbids any allocation afterwards.  Such a
 // caller cannot provide the workspace csa_decode needs for its split-K
 // partial results.  This entry point runs the same decode kernel, but its
-// scratch (flag word, merge tickets and partial records) lives in one
+// scratch (flag word, record ranges and partial records) lives in one
 // file-scope __device__ array of kNoAllocScratchBytes that every GPU which
 // loads the library keeps until the process exits.  The call itself
 // allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
@@ -18,8 +18,9 @@
 // call before any stream capture.
 //
 // All calls share the one array and it keeps whatever the previous call left:
-// the flag word and the tickets are cleared on the caller's stream at the
-// start of every call; the partial records need no clearing.  Two calls whose
+// the flag word is cleared on the caller's stream at the start of every call;
+// the record ranges and partial records are rewritten by every call before
+// they are read.  Two calls whose
 // kernels overlap on a GPU therefore race on the array: issue them on one
 // stream, or order them.
 #include <math.h>
@@ -50,42 +51,6 @@ void* scratch_address(int dev) {
         g_scratch_addr[dev] = p;
     }
     return g_scratch_addr[dev];
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-        else
-            cudaGetLastError();
-    });
-    return fn;
-}
-
-// Same view of a paged cache as csa_decode uses: [num_pages * Hkv * 16][D]
-// bf16, 64-channel x 16-token boxes, 128-byte swizzle.
-bool cache_map(CUtensorMap* m, const void* base, const Shape& s) {
-    EncodeTiledFn fn = encode_tiled();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)s.D, (cuuint64_t)s.NPG * s.Hkv * kPage};
-    cuuint64_t strides[1] = {(cuuint64_t)s.D * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kPage};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
 }
 
 bool ok16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
@@ -127,12 +92,12 @@ extern "C" int csa_decode_noalloc(const csa_dims* d, const void* q, const void* 
     s.NPG = d->num_pages;
     s.max_sel = d->max_sel;
 
-    // scratch: [flag word | tickets | partial records], each 256-byte aligned
+    // scratch: [flag word | record ranges | partial records], each 256-byte aligned
     const size_t units = (size_t)s.B * s.Hkv;
-    const size_t tickets_off = 256;
-    const size_t partials_off = tickets_off + up256(4 * units);
+    const size_t ranges_off = 256;
+    const size_t partials_off = ranges_off + up256(8 * units);
     const size_t slots = (size_t)decode_grid(s) + units;
-    const size_t need = partials_off + 4 * slots * (size_t)G * (s.D + 2);
+    const size_t need = partials_off + 4 * slots * decode_record_floats(s);
     if (need > kNoAllocScratchBytes) return CSA_ERR_WORKSPACE;   // shape needs more scratch
 
     int dev = 0;
@@ -143,16 +108,15 @@ extern "C" int csa_decode_noalloc(const csa_dims* d, const void* q, const void* 
     uint8_t* scratch = static_cast<uint8_t*>(scratch_address(dev));
     if (!scratch) return CSA_ERR_CUDA;
 
-    CUtensorMap tmK, tmV;
-    if (!cache_map(&tmK, k_cache, s) || !cache_map(&tmV, v_cache, s)) return CSA_ERR_CUDA;
-
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemsetAsync(scratch, 0, partials_off, st) != cudaSuccess) {   // flag + tickets
+    if (cudaMemsetAsync(scratch, 0, 4, st) != cudaSuccess) {   // flag word
         cudaGetLastError();
         return CSA_ERR_CUDA;
     }
     DecodeParams p;
     p.q = static_cast<const uint16_t*>(q);
+    p.k_cache = static_cast<const uint16_t*>(k_cache);
+    p.v_cache = static_cast<const uint16_t*>(v_cache);
     p.page_table = page_table;
     p.seq_lens = seq_lens;
     p.sel = sel_pages;
@@ -165,10 +129,10 @@ extern "C" int csa_decode_noalloc(const csa_dims* d, const void* q, const void* 
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
     p.flags = reinterpret_cast<uint32_t*>(scratch);
-    p.tickets = reinterpret_cast<uint32_t*>(scratch + tickets_off);
+    p.rec_range = reinterpret_cast<int2*>(scratch + ranges_off);
     p.partials = reinterpret_cast<float*>(scratch + partials_off);
     p.s = s;
-    if (launch_decode(p, tmK, tmV, st) != cudaSuccess) {
+    if (launch_decode(p, st) != cudaSuccess) {
         cudaGetLastError();
         return CSA_ERR_CUDA;
     }

@@ -13,16 +13,21 @@
 // are exact in fp32; fp32 accumulation), and the kv-head score is the max
 // over the group's heads.
 //
-// Data path (the kernel is HBM-bound: it streams 4*D bytes of metadata per
-// candidate page and does ~2 flop per byte):
+// Data path.  The kernel streams 4*D bytes of metadata per candidate page
+// from random physical pages and does ~2 flop per byte: it is HBM-bound, and
+// what decides its speed is how many bytes are in flight.  Every warp of the
+// grid loads its own tiles straight into the registers that feed the MMA:
+// with the k index of the contraction permuted (the same permutation on the
+// q side), lane (g, t) of a warp needs exactly the 16-byte chunks
+// t, t+4, t+8, ... of rows g and g+8 of the tile, so a tile is 2D/16 plain
+// 16-byte loads per lane (non-allocating in L1), with no shared-memory
+// staging and no barriers.  Measured on B200 for 16 x 512-byte rows this
+// sustains ~81% of the copy peak, where a TMA bulk copy per row (512 bytes)
+// is limited by its per-copy issue cost to ~30%.
 //   * the candidates of all (sequence, kv-head) units are flattened and split
-//     evenly over a grid sized to fill every SM;
+//     evenly over a grid that fills every SM;
 //   * each CTA copies its slice of the page table into shared memory once;
-//   * a producer warp issues one TMA bulk copy (cp.async.bulk) per page into
-//     a ring of 16-page stages tracked by mbarriers with byte counts; rows are
-//     padded to 4*D+16 bytes so that the fragment loads are bank-conflict free;
-//   * four consumer warps each take whole stages: 2D/16 mma.sync m16n8k16 per
-//     tile, a quad-shuffle max over heads, fp32 scores out.
+//   * warps take the CTA's 16-page tiles round-robin.
 #include "common.cuh"
 #include "internal.h"
 
@@ -31,21 +36,12 @@ namespace {
 
 template <int D, int NB>
 struct ScoreCfg {
-    static constexpr int kConsumers = 4;
-    static constexpr int kThreads = 32 * (kConsumers + 1);
-    static constexpr int kTile = 16;                  // pages per stage (one m16 tile)
-    static constexpr int kRowBytes = 4 * D;           // [min | max] bf16 of one (page, kv-head)
-    static constexpr int kRowStride = 4 * D + 16;     // padded shared-memory row
-    static constexpr int kStageBytes = kTile * kRowStride;
-    static constexpr int kStages = D >= 256 ? 4 : 8;
-    // a stage's previous use must belong to the same consumer warp, so that a
-    // parity wait can never be two phases ahead of the barrier
-    static_assert(kStages % kConsumers == 0, "stages must be a multiple of consumers");
+    static constexpr int kWarps = 8;
+    static constexpr int kThreads = 32 * kWarps;
     static constexpr int kKPairs = 2 * D / 32;        // 32-channel steps along [min | max]
-    // stages | page-table slice | full/empty barriers | tile infos | 3 x [B + 1] ints
+    // page-table slice | 3 x [B + 1] ints
     static __host__ __device__ size_t smem_bytes(int B) {
-        return (size_t)kStages * kStageBytes + (size_t)kScorePtCap * 4 + 16 * (size_t)kStages +
-               16 * (size_t)kStages + 3 * 4 * (size_t)(B + 1);
+        return (size_t)kScorePtCap * 4 + 3 * 4 * (size_t)(B + 1);
     }
 };
 
@@ -53,7 +49,6 @@ struct TileInfo {
     int unit;      // b * Hkv + g
     int first;     // logical page of row 0
     int count;     // rows in use (1..16)
-    uint32_t valid;
 };
 
 __device__ __forceinline__ uint32_t neg_part(uint32_t w) {   // min(q, 0) per bf16 half
@@ -120,130 +115,29 @@ struct TileWalker {
     }
 };
 
-// After a timed-out wait (the CTA unwinds with CSA_DEVFLAG_TIMEOUT latched),
-// keep the CTA alive, again for a bounded time, until every copy it issued
-// has landed, so that no TMA write targets shared memory of a finished CTA.
-template <int kStages>
-__device__ void drain_issued(uint64_t* full, int issued) {
-    for (int st = 0; st < kStages && st < issued; ++st) {
-        const int last = st + ((issued - 1 - st) / kStages) * kStages;   // last use of st
-        mbar_wait(&full[st], (last / kStages) & 1);
-    }
-}
-
-// Consumer warps: score whole 16-page stages on the tensor cores.
-template <int D, int NB>
-__device__ __forceinline__ void consume(const ScoreParams& p, TileWalker walk, uint8_t* stages,
-                                        uint64_t* full, uint64_t* empty, const TileInfo* info,
-                                        int* s_abort, int warp, int lane) {
-    using C = ScoreCfg<D, NB>;
-    const int Hkv = p.s.Hkv, G = p.s.G, MP = p.s.MP;
-    const int gq = lane >> 2, tq = lane & 3;
-    uint32_t qf[C::kKPairs][NB][4];          // B fragments of [q- | q+] for the current unit
-    int cur_unit = -1;
-    TileInfo t;
-    for (int j = 0; walk.next(t); ++j) {
-        if (j % C::kConsumers != warp) continue;
-        const int st = j % C::kStages;
-        const int r = j / C::kStages;
-        if (!mbar_wait(&full[st], r & 1)) {
-            if (lane == 0) latch_flag(p.flags, CSA_DEVFLAG_TIMEOUT);
-            *s_abort = 1;
-            break;
-        }
-        if (*(volatile int*)s_abort) break;
-        const TileInfo ti = info[st];
-        if (ti.unit != cur_unit) {
-            cur_unit = ti.unit;
-            const int b = ti.unit / Hkv, g = ti.unit % Hkv;
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const int head = nb * 8 + gq;
-                const uint32_t* qw = reinterpret_cast<const uint32_t*>(
-                    p.q + ((size_t)b * p.s.Hq + (size_t)g * G + head) * D);
-#pragma unroll
-                for (int kp = 0; kp < C::kKPairs; ++kp) {
-                    // channels ch0 .. ch0+7 of the [min | max] row; min pairs with q-
-                    const int ch0 = 32 * kp + 8 * tq;
-                    const bool is_max = ch0 >= D;
-                    const int qc = is_max ? ch0 - D : ch0;
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        uint32_t v = head < G ? __ldg(qw + qc / 2 + w) : 0u;
-                        qf[kp][nb][w] = is_max ? pos_part(v) : neg_part(v);
-                    }
-                }
-            }
-        }
-        float acc[NB][4];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-            acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-        const uint32_t base = smem_u32(stages + (size_t)st * C::kStageBytes);
-        const uint32_t row0 = base + gq * C::kRowStride + 16 * tq;
-        const uint32_t row8 = row0 + 8 * C::kRowStride;
-#pragma unroll
-        for (int kp = 0; kp < C::kKPairs; ++kp) {
-            const uint4 x = ld_shared_v4(row0 + 64 * kp);
-            const uint4 y = ld_shared_v4(row8 + 64 * kp);
-            const uint32_t a0[4] = {x.x, y.x, x.y, y.y};
-            const uint32_t a1[4] = {x.z, y.z, x.w, y.w};
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                mma_bf16_16816(acc[nb], a0, qf[kp][nb][0], qf[kp][nb][1]);
-                mma_bf16_16816(acc[nb], a1, qf[kp][nb][2], qf[kp][nb][3]);
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);   // stage free once fragments are loaded
-        // max over the group's heads: this lane holds heads 8nb + 2tq, +1
-        float m0 = -INFINITY, m8 = -INFINITY;
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-            const int h = nb * 8 + 2 * tq;
-            if (h < G) {
-                m0 = fmaxf(m0, acc[nb][0]);
-                m8 = fmaxf(m8, acc[nb][2]);
-            }
-            if (h + 1 < G) {
-                m0 = fmaxf(m0, acc[nb][1]);
-                m8 = fmaxf(m8, acc[nb][3]);
-            }
-        }
-        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-        m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
-        m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
-        const int row = tq == 0 ? gq : gq + 8;
-        if (tq < 2 && row < ti.count) {
-            float v = tq == 0 ? m0 : m8;
-            if (!((ti.valid >> row) & 1u)) v = -INFINITY;
-            const size_t o = (size_t)ti.unit * MP + ti.first + row;
-            p.scores_ws[o] = v;
-            if (p.scores_out) p.scores_out[o] = v;
-        }
-    }
+// 16-byte load that does not allocate in L1 (the metadata is read once).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
 }
 
 template <int D, int NB>
 __global__ void __launch_bounds__(ScoreCfg<D, NB>::kThreads)
 score_kernel(ScoreParams p) {
     using C = ScoreCfg<D, NB>;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    uint8_t* stages = smem;
-    int* pt = reinterpret_cast<int*>(stages + (size_t)C::kStages * C::kStageBytes);
-    uint64_t* full = reinterpret_cast<uint64_t*>(pt + kScorePtCap);
-    uint64_t* empty = full + C::kStages;
-    TileInfo* info = reinterpret_cast<TileInfo*>(empty + C::kStages);
-    int* seq_n = reinterpret_cast<int*>(info + C::kStages);
+    extern __shared__ __align__(16) int smem_i[];
+    int* pt = smem_i;
+    int* seq_n = pt + kScorePtCap;
     int* seq_clo = seq_n + (p.s.B + 1);
     int* seq_off = seq_clo + (p.s.B + 1);
-    __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.s.B, Hkv = p.s.Hkv, G = p.s.G, MP = p.s.MP;
 
-    // Candidates per sequence.
+    // Candidates per sequence (caller inputs only before the dependency wait).
     for (int b = tid; b < B; b += C::kThreads) {
         int L = p.seq_lens[b];
         if (L < 0 || L > MP * kPage) {
@@ -254,7 +148,6 @@ score_kernel(ScoreParams p) {
         seq_n[b] = sg.c_hi - sg.c_lo;
         seq_clo[b] = sg.c_lo;
     }
-    if (tid == 0) s_abort = 0;
     __syncthreads();
     if (warp == 0) {   // exclusive scan of Hkv * n_b
         int carry = 0;
@@ -274,24 +167,19 @@ score_kernel(ScoreParams p) {
     }
     __syncthreads();
     const long long N = seq_off[B];
-    const long long s = N * blockIdx.x / gridDim.x, e = N * (blockIdx.x + 1) / gridDim.x;
-    if (s >= e) {
-        pdl_wait();
-        pdl_launch_dependents();
-        return;
-    }
+    const int s = (int)(N * blockIdx.x / gridDim.x), e = (int)(N * (blockIdx.x + 1) / gridDim.x);
 
-    // Page-table slice of this CTA (the grid is sized so that e - s <= cap),
-    // copied run by run: every run is a contiguous piece of one page-table row.
     TileWalker walk;
     walk.seq_off = seq_off;
     walk.seq_n = seq_n;
     walk.seq_clo = seq_clo;
     walk.Hkv = Hkv;
     walk.B = B;
-    {
+    if (s < e) {
+        // page-table slice (the grid is sized so that e - s <= cap), run by run:
+        // every run is a contiguous piece of one page-table row
         TileWalker fill = walk;
-        fill.start((int)s, (int)e);
+        fill.start(s, e);
         TileInfo run;
         int at = 0;
         while (fill.next(run, 1 << 30)) {
@@ -300,61 +188,98 @@ score_kernel(ScoreParams p) {
             at += run.count;
         }
     }
-    walk.start((int)s, (int)e);
-    __shared__ int s_issued;
-    if (tid == 0) {
-        for (int i = 0; i < C::kStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-        }
-        fence_barrier_init();
-        s_issued = 0;
-    }
     // the metadata was written by the previous kernel on the stream
     pdl_wait();
     pdl_launch_dependents();
     __syncthreads();
+    if (s >= e) return;
 
-    if (warp == C::kConsumers) {
-        // ------------------------------------------------------------ producer
-        TileInfo t;
-        for (int j = 0; walk.next(t); ++j) {
-            const int st = j % C::kStages;
-            const int r = j / C::kStages;
-            if (lane == 0 && r > 0 && !mbar_wait(&empty[st], (r - 1) & 1)) {
-                latch_flag(p.flags, CSA_DEVFLAG_TIMEOUT);
-                s_abort = 1;
-            }
-            __syncwarp();
-            if (*(volatile int*)&s_abort) break;
-            const int g = t.unit % Hkv;
-            const int x0 = walk.x - t.count - (int)s;    // slice index of row 0
-            int phys = -1;
-            bool ok = false;
-            if (lane < t.count) {
-                phys = pt[x0 + lane];
-                ok = phys >= 0 && phys < p.s.NPG;
-                if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
-            }
-            const uint32_t valid = __ballot_sync(0xffffffffu, ok);
-            if (lane == 0) {
-                t.valid = valid;
-                info[st] = t;
-                mbar_arrive_expect_tx(&full[st], (uint32_t)__popc(valid) * C::kRowBytes);
-            }
-            __syncwarp();
-            if (ok) {
-                const uint16_t* src = p.meta + ((size_t)phys * Hkv + g) * 2 * D;
-                tma_bulk_g2s(stages + (size_t)st * C::kStageBytes + lane * C::kRowStride, src,
-                             C::kRowBytes, &full[st]);
-            }
-            if (lane == 0) s_issued = j + 1;
+    const int gq = lane >> 2, tq = lane & 3;
+    uint32_t qf[C::kKPairs][NB][4];          // B fragments of [q- | q+] for the current unit
+    int cur_unit = -1;
+    walk.start(s, e);
+    TileInfo t;
+    for (int j = 0; walk.next(t); ++j) {
+        if (j % C::kWarps != warp) continue;
+        const int b = t.unit / Hkv, g = t.unit % Hkv;
+        const int x0 = walk.x - t.count - s;           // slice index of row 0
+        // rows g and g+8 of the tile (clamped inside the tile; extra rows are dropped)
+        const int r0 = gq < t.count ? gq : t.count - 1;
+        const int r8 = gq + 8 < t.count ? gq + 8 : t.count - 1;
+        const int p0 = pt[x0 + r0], p8 = pt[x0 + r8];
+        const bool ok0 = p0 >= 0 && p0 < p.s.NPG, ok8 = p8 >= 0 && p8 < p.s.NPG;
+        const char* row0 = reinterpret_cast<const char*>(
+            p.meta + ((size_t)(ok0 ? p0 : 0) * Hkv + g) * 2 * D) + 16 * tq;
+        const char* row8 = reinterpret_cast<const char*>(
+            p.meta + ((size_t)(ok8 ? p8 : 0) * Hkv + g) * 2 * D) + 16 * tq;
+        uint4 xa[C::kKPairs], xb[C::kKPairs];
+#pragma unroll
+        for (int kp = 0; kp < C::kKPairs; ++kp) {
+            xa[kp] = ld_stream_v4(row0 + 64 * kp);
+            xb[kp] = ld_stream_v4(row8 + 64 * kp);
         }
-    } else {
-        consume<D, NB>(p, walk, stages, full, empty, info, &s_abort, warp, lane);
+        if (t.unit != cur_unit) {
+            cur_unit = t.unit;
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int head = nb * 8 + gq;
+                const uint32_t* qw = reinterpret_cast<const uint32_t*>(
+                    p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
+#pragma unroll
+                for (int kp = 0; kp < C::kKPairs; ++kp) {
+                    // channels ch0 .. ch0+7 of the [min | max] row; min pairs with q-
+                    const int ch0 = 32 * kp + 8 * tq;
+                    const bool is_max = ch0 >= D;
+                    const int qc = is_max ? ch0 - D : ch0;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const uint32_t v = head < G ? __ldg(qw + qc / 2 + w) : 0u;
+                        qf[kp][nb][w] = is_max ? pos_part(v) : neg_part(v);
+                    }
+                }
+            }
+        }
+        float acc[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+#pragma unroll
+        for (int kp = 0; kp < C::kKPairs; ++kp) {
+            const uint32_t a0[4] = {xa[kp].x, xb[kp].x, xa[kp].y, xb[kp].y};
+            const uint32_t a1[4] = {xa[kp].z, xb[kp].z, xa[kp].w, xb[kp].w};
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                mma_bf16_16816(acc[nb], a0, qf[kp][nb][0], qf[kp][nb][1]);
+                mma_bf16_16816(acc[nb], a1, qf[kp][nb][2], qf[kp][nb][3]);
+            }
+        }
+        // max over the group's heads: this lane holds heads 8nb + 2tq, +1
+        float m0 = -INFINITY, m8 = -INFINITY;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            const int h = nb * 8 + 2 * tq;
+            if (h < G) {
+                m0 = fmaxf(m0, acc[nb][0]);
+                m8 = fmaxf(m8, acc[nb][2]);
+            }
+            if (h + 1 < G) {
+                m0 = fmaxf(m0, acc[nb][1]);
+                m8 = fmaxf(m8, acc[nb][3]);
+            }
+        }
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+        m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
+        m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
+        const int row = tq == 0 ? gq : gq + 8;
+        if (tq < 2 && row < t.count) {
+            const bool ok = tq == 0 ? ok0 : ok8;
+            if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
+            const float v = ok ? (tq == 0 ? m0 : m8) : -INFINITY;
+            const size_t o = (size_t)t.unit * MP + t.first + row;
+            p.scores_ws[o] = v;
+            if (p.scores_out) p.scores_out[o] = v;
+        }
     }
-    __syncthreads();
-    if (tid == 0 && s_abort) drain_issued<C::kStages>(full, s_issued);
 }
 
 template <int D, int NB>
@@ -371,16 +296,12 @@ cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t st) {
         attr_done[dev] = 1;
     }
     const size_t smem = C::smem_bytes(p.s.B);
-    // resident CTAs per SM: registers allow several; shared memory decides
-    int occ = (int)((size_t)(228 * 1024) / (smem + 1024));
-    if (occ > 4) occ = 4;
-    if (occ < 1) occ = 1;
     const long long ub = (long long)p.s.B * p.s.Hkv * p.s.MP;
-    long long grid = (long long)occ * device_sm_count();
+    long long grid = 2LL * device_sm_count();      // two resident CTAs of 8 warps per SM
     const long long need = (ub + kScorePtCap - 1) / kScorePtCap;
     if (need > grid) grid = need;
     if (grid < 1) grid = 1;
-    return launch_pdl(score_kernel<D, NB>, dim3((unsigned)grid), dim3(C::kThreads), smem, st, p);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(C::kThreads), smem, st, p);
 }
 
 }  // namespace
