@@ -69,18 +69,23 @@ def parse_args():
 
 # ---------------------------------------------------------------- plumbing
 class Dist:
-    def __init__(self):
+    """One process per GPU (torchrun's RANK/LOCAL_RANK/WORLD_SIZE); the only
+    collectives are the timing barrier and the max over ranks."""
+
+    def __init__(self, backend: str | None = None, timeout_s: float = 180.0):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.backend = None
         if self.world > 1:
             import torch.distributed as dist
-            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
             if backend == "nccl":
                 torch.cuda.set_device(self.local)
-            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
             self.pg = dist
+            self.backend = backend
 
     def barrier(self):
         if self.pg:
@@ -89,7 +94,7 @@ class Dist:
     def max(self, x: float) -> float:
         if not self.pg:
             return x
-        dev = torch.device("cuda", self.local) if torch.cuda.is_available() else "cpu"
+        dev = torch.device("cuda", self.local) if self.backend == "nccl" else "cpu"
         t = torch.tensor([x], dtype=torch.float64, device=dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
@@ -97,6 +102,18 @@ class Dist:
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def rank_workload(base: wl.Workload, rank: int, total_steps: int) -> wl.Workload:
+    """The replica a rank decodes: the same shapes as `base`, its own seed.
+    Ranks share nothing, so the path needs no collective (weak scaling)."""
+    return replace(base, steps=total_steps, seed=base.seed + 1000 * rank)
+
+
+def job_value(world: int, units_per_rank: int, t_max: float) -> float:
+    """Whole-job throughput: units every rank processed over the slowest
+    rank's device time."""
+    return world * units_per_rank / t_max
 
 
 def score_traffic():
@@ -221,10 +238,10 @@ def run_reference(args, dist: Dist, w: wl.Workload):
 class Stack:
     """All layers of a workload on one GPU, with per-step inputs resident."""
 
-    def __init__(self, w: wl.Workload, dev, total_steps: int, seed_offset: int):
+    def __init__(self, w: wl.Workload, dev):
         from long_context_decoding_b200 import csa
         self.csa = csa
-        self.w = w = replace(w, steps=total_steps, seed=w.seed + seed_offset)
+        self.w = w
         self.dev = dev
         self.d = csa.make_dims(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.num_pages, w.max_sel)
         self.ws = csa.new_workspace(self.d, dev)
@@ -237,9 +254,9 @@ class Stack:
             lay.case = c
             self.layers.append(lay)
         L0 = torch.tensor(w.seq_lens, dtype=torch.int32, device=dev)
-        self.lens = [(L0 + s + 1).contiguous() for s in range(total_steps)]
+        self.lens = [(L0 + s + 1).contiguous() for s in range(w.steps)]
         self.inputs = [[wl.step_tokens(lay.case, s) for lay in self.layers]
-                       for s in range(total_steps)]
+                       for s in range(w.steps)]
         torch.cuda.synchronize()
         assert csa.device_status(self.ws) == 0
 
@@ -263,9 +280,11 @@ class Stack:
                            lay.n_sel, lay.prefix, lay.window, lay.out, self.ws, lay.lse)
 
     def launches_per_step(self) -> int:
+        """Kernels of one step: per layer meta update, score (only when pages
+        are selected), select, decode and its split-K combine."""
         n = 0
         for lay in self.layers:
-            n += 1 + 1 + (1 if lay.budget // 16 > 0 else 0) + 1
+            n += 1 + (1 if lay.budget // 16 > 0 else 0) + 1 + 2
         return n
 
     def graph(self, fn):
@@ -303,7 +322,7 @@ def run_ours(args, dist: Dist, base: wl.Workload):
     dev = torch.device("cuda", dist.local)
     torch.cuda.set_device(dev)
     K, W = args.steps, args.warmup
-    st = Stack(base, dev, K + W, seed_offset=1000 * dist.rank)
+    st = Stack(rank_workload(base, dist.rank, K + W), dev)
     w = st.w
     nl = len(st.layers)
     # eager pass over every step: sets kernel attributes, checks the flags
@@ -328,7 +347,7 @@ def run_ours(args, dist: Dist, base: wl.Workload):
     clk = clocks.stop() if clocks else None
     t = dist.max(t)
     flags = st.csa.device_status(st.ws)
-    value = dist.world * w.B * nl * K / t
+    value = job_value(dist.world, w.B * nl * K, t)
     t_layer = t / (K * nl)
 
     # per-layer algorithmic bytes over the timed steps (averaged)

@@ -47,12 +47,24 @@
  *
  * ----------------------------------------------------------- conventions
  *  - Every pointer argument except the ones marked "host" is a DEVICE
- *    pointer owned by the caller; the library allocates no memory and holds
- *    no per-call state outside the caller's workspace.
+ *    pointer owned by the caller; the library allocates no device memory.
  *  - Device pointers must be 16-byte aligned (CSA_ERR_INVALID_ARG if not).
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All calls
  *    are asynchronous on it; the status code reports argument checks and
  *    launch errors only.  Calls sharing one workspace must not overlap.
+ *  - Kernels are launched with programmatic dependent launch, so a kernel
+ *    may start while the previous kernel on the stream finishes.  Each call
+ *    waits for the preceding work before it reads anything, with two
+ *    exceptions.  (1) csa_score_select reads `page_table` and `seq_lens`
+ *    early: those two must not come from the kernel launched just before the
+ *    call if that kernel releases its dependents early (a host copy, an
+ *    event, a plain kernel or a call of this library is fine).  (2) When the
+ *    previous call of this library on the same stream was csa_score_select,
+ *    csa_decode / csa_decode_full stream the prefix and window pages while
+ *    the selection kernel is still running: their `q`, `k_cache`,
+ *    `v_cache`, `page_table` and `seq_lens` must not be written between the
+ *    two calls.  The library remembers the last call per stream handle on
+ *    the host; this is its only state outside the workspace.
  *  - Page ids that fall outside [0, num_pages), selected pages outside the
  *    candidate range, and a selection that is not strictly ascending are
  *    detected on the device: the page is skipped and a flag is latched in
@@ -88,7 +100,7 @@ enum {
                                      not ascending, or n_sel out of range     */
     CSA_DEVFLAG_BAD_SEQ_LEN = 4,  /* seq_len < 0 or > 16 * max_pages_per_seq,
                                      or shorter than the appended chunk       */
-    CSA_DEVFLAG_TIMEOUT = 8       /* a bounded pipeline wait gave up          */
+    CSA_DEVFLAG_TIMEOUT = 8       /* reserved: no kernel of this version waits */
 };
 
 /* Problem shape, passed by host pointer to every call. */

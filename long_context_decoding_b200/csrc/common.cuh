@@ -1,15 +1,12 @@
 // common.cuh -- device helpers shared by the libcsa kernels (sm_100a).
 //
-// Thin inline-PTX wrappers for the Hopper/Blackwell async machinery the
-// kernels are built on: mbarrier phases with transaction counts, the TMA
-// engine (1-D bulk copies and 2-D tensor tiles with 128-byte swizzle), the
-// warp-level bf16 tensor-core MMA, ldmatrix / movmatrix fragment moves and
-// programmatic dependent launch.  Every wait here is bounded in time: when
-// the bound runs out the caller latches CSA_DEVFLAG_TIMEOUT and unwinds, so
-// no kernel can spin forever.
+// bf16 bit helpers, an order-preserving float -> key map, inline-PTX wrappers
+// for the warp-level bf16 tensor-core MMA and the ldmatrix / movmatrix
+// fragment moves, programmatic dependent launch, and the per-sequence token
+// geometry (prefix, window, candidate pages) every kernel shares.  No kernel
+// of the library spins on a flag or barrier of its own.
 #pragma once
 
-#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -24,7 +21,6 @@ constexpr int kPage = 16;                       // tokens per page
 constexpr int kMaxUnits = 2048;                 // B * Hkv supported per call
 constexpr int kScorePtCap = 4096;               // page-table entries staged per scoring CTA
 constexpr int kDecodeItemCap = 1024;            // pages staged per decode CTA
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
 // ------------------------------------------------------------ bf16 / keys
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -52,12 +48,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ unsigned long long global_timer_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
 __device__ __forceinline__ float ex2(float x) {     // 2^x, hardware approximation
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -73,74 +63,6 @@ __device__ __forceinline__ void latch_flag(uint32_t* flags, uint32_t bit) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// ------------------------------------------------------------ mbarrier
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-                 : "memory");
-}
-// Make barrier initialisation visible to the async (TMA) proxy.
-__device__ __forceinline__ void fence_barrier_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-// Order this thread's generic-proxy shared-memory accesses before later
-// async-proxy (TMA) accesses to the same memory.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
-                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Wait for phase `parity` of `bar` to complete; false after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_timer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
-    }
-}
-
-// ------------------------------------------------------------ TMA
-// 1-D bulk copy global -> shared, completion counted on `bar` (bytes).
-// dst, src 16-byte aligned; bytes a multiple of 16.
-__device__ __forceinline__ void tma_bulk_g2s(void* dst, const void* src, uint32_t bytes,
-                                             uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-// 2-D tensor tile global -> shared (layout and swizzle from the tensor map).
-// c0 is the innermost (element) coordinate; callers keep it 16-byte aligned.
-__device__ __forceinline__ void tma_tile_g2s(void* dst, const CUtensorMap* map, int c0, int c1,
-                                             uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1),
-          "r"(smem_u32(bar))
-        : "memory");
-}
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // ------------------------------------------------------------ tensor core
@@ -177,15 +99,6 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
     return d;
 }
 
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-
 // ------------------------------------------------------------ sequence geometry
 // Token ranges of one sequence for one call: effective prefix Pe and window
 // We, logical pages np, and the top-k candidate pages [c_lo, c_hi): the
@@ -216,6 +129,7 @@ __host__ __device__ __forceinline__ SeqGeom seq_geom(int L, int prefix, int wind
 // library therefore reads only caller inputs before pdl_wait(), and calls
 // pdl_launch_dependents() only after it, so that when a kernel starts, all
 // kernels two or more launches earlier have completed.
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t st, Args&&... args) {

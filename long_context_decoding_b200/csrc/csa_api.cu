@@ -1,12 +1,13 @@
 // csa_api.cu -- the C ABI of libcsa.so (declared in include/csa.h).
 //
-// Host-side only: argument validation, the workspace layout, TMA tensor-map
-// encoding and kernel dispatch.  No memory is allocated here; every buffer
-// belongs to the caller.
+// Host-side only: argument validation, the workspace layout, the per-stream
+// record of the last call and kernel dispatch.  No device memory is
+// allocated here; every buffer belongs to the caller.
 #include <math.h>
 #include <mutex>
 #include <stdio.h>
 #include <string.h>
+#include <unordered_map>
 
 #include "common.cuh"
 #include "internal.h"
@@ -33,21 +34,37 @@ int device_sm_count() {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Last kernel-launching call per stream handle.  Forgetting an entry is
+// always safe (the decode then waits before it reads anything), so the table
+// is simply cleared when it grows large.
+static std::mutex g_calls_mu;
+static std::unordered_map<const void*, CallKind> g_calls;
+
+void note_stream_call(const void* stream, CallKind kind) {
+    std::lock_guard<std::mutex> lock(g_calls_mu);
+    if (g_calls.size() > 4096) g_calls.clear();
+    g_calls[stream] = kind;
+}
+
+CallKind last_stream_call(const void* stream) {
+    std::lock_guard<std::mutex> lock(g_calls_mu);
+    auto it = g_calls.find(stream);
+    return it == g_calls.end() ? kCallOther : it->second;
+}
+
 WsLayout workspace_layout(const Shape& s) {
     WsLayout w;
     const size_t units = (size_t)s.B * s.Hkv;
     size_t off = 0;
     w.flags = off;
     off = align_up(off + 4, 256);
-    w.score_tickets = off;
-    off = align_up(off + 4 * units, 256);
     w.rec_range = off;
-    off = align_up(off + 8 * units, 256);
+    off = align_up(off + 16 * units, 256);
     w.scores = off;
     off = align_up(off + 4 * units * (size_t)s.MP, 256);
     w.partials = off;
     w.dec_slots = (size_t)decode_grid(s) + units;
-    off = align_up(off + 4 * w.dec_slots * decode_record_floats(s), 256);
+    off = align_up(off + 2 * 4 * w.dec_slots * decode_record_floats(s), 256);
     w.total = off;
     return w;
 }
@@ -172,6 +189,7 @@ int csa_meta_update(const csa_dims* d, void* k_cache, void* v_cache, void* meta,
     p.n_new = n_new;
     p.flags = at<uint32_t>(workspace, w.flags);
     p.s = s;
+    note_stream_call(stream, kCallOther);
     return launch_status(launch_meta_update(p, (cudaStream_t)stream));
 }
 
@@ -209,7 +227,10 @@ int csa_score_select(const csa_dims* d, const void* q, const void* meta,
     sp.s = s;
     if (k_pages > 0 || scores_out) {
         rc = launch_status(launch_score(sp, st));
-        if (rc != CSA_OK) return rc;
+        if (rc != CSA_OK) {
+            note_stream_call(stream, kCallOther);
+            return rc;
+        }
     }
     SelectParams lp;
     lp.scores_ws = sp.scores_ws;
@@ -222,7 +243,9 @@ int csa_score_select(const csa_dims* d, const void* q, const void* meta,
     lp.flags = sp.flags;
     lp.smem_keys = 0;
     lp.s = s;
-    return launch_status(launch_select(lp, st));
+    rc = launch_status(launch_select(lp, st));
+    note_stream_call(stream, rc == CSA_OK ? kCallScoreSelect : kCallOther);
+    return rc;
 }
 
 static int decode_common(const csa_dims* d, const void* q, const void* k_cache,
@@ -265,9 +288,12 @@ static int decode_common(const csa_dims* d, const void* q, const void* k_cache,
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
     p.flags = at<uint32_t>(workspace, w.flags);
-    p.rec_range = at<int2>(workspace, w.rec_range);
+    p.rec_range = at<int4>(workspace, w.rec_range);
     p.partials = at<float>(workspace, w.partials);
+    p.phase_floats = w.dec_slots * decode_record_floats(s);
+    p.early = last_stream_call(stream) == kCallScoreSelect ? 1 : 0;
     p.s = s;
+    note_stream_call(stream, kCallOther);
     return launch_status(launch_decode(p, (cudaStream_t)stream));
 }
 

@@ -1,5 +1,5 @@
-// decode.cu -- split-K flash decoding over the attended pages, with the
-// cross-CTA merge fused in ("last CTA per unit combines").
+// decode.cu -- split-K flash decoding over the attended pages, in two phases,
+// and the kernel that merges the split results.
 //
 // Combined sparse attention ("Accelerating Long-Context Decoding in
 // Large-Scale Hybrid LLMs Without Retraining", abstract): every query head
@@ -8,23 +8,23 @@
 //     A = { t < L : t < Pe  or  t >= L - We  or  page(t) selected }
 // and for each of the G query heads of the group
 //     out_h = sum_{t in A} softmax_t(scale * q_h . k_t) v_t .
-// The dense layer (csa_decode_full) is the same kernel with every page
-// selected.
+// The dense layer (csa_decode_full) is the same kernel with every page fixed.
 //
-// Work list.  Per unit the pages to read are, in order: the prefix-only
-// pages [0, c_lo), the prefix boundary page c_lo when it is not selected but
-// holds prefix tokens, the selected pages, the window boundary page c_hi - 1
-// when it is not selected but holds window tokens, and the window-only pages
-// [c_hi, np).  A token mask (t < L and (selected-page or t < Pe or
-// t >= L - We)) makes the union token-exact with nothing counted twice.  The
-// lists of all units are flattened and split evenly over a grid that fills
-// every SM, so ragged lengths and budgets stay balanced.
+// Two phases.  Phase 0 takes the fixed list of every unit: the pages holding
+// prefix or window tokens, masked to those tokens.  Phase 1 takes the
+// selected pages, masked to their other tokens (a selected boundary page is
+// split between the phases, so the union is token-exact and nothing counts
+// twice).  Phase 0 does not depend on the selection: when the call follows
+// csa_score_select on the same stream it runs before the dependency wait,
+// while the selection kernel is still working, and only phase 1 waits.  In
+// each phase the lists of all units are flattened and split evenly over the
+// grid, so ragged lengths and budgets stay balanced.
 //
-// Per CTA: the page ids of its slice are resolved once into shared memory;
-// every warp then streams its own pages (round-robin over the slice) with
-// 16-byte cp.async copies into a private double buffer, laid out with the
-// 128-byte XOR swizzle (16-byte chunk c of token row r at c ^ (r & 7)), so
-// ldmatrix reads it without bank conflicts; slots past the end of the
+// Per CTA and phase: the page ids of its slice are resolved once into shared
+// memory; every warp then streams its own pages (round-robin over the slice)
+// with 16-byte cp.async copies into a private double buffer, laid out with
+// the 128-byte XOR swizzle (16-byte chunk c of token row r at c ^ (r & 7)),
+// so ldmatrix reads it without bank conflicts; slots past the end of the
 // sequence are zero-filled by the copy itself.  (Per-page TMA copies were
 // measured slower here: their issue cost, paid serially by one thread, caps
 // a CTA's request rate.)  Per page a warp computes S^T = K Q^T (16 tokens x
@@ -32,9 +32,9 @@
 // resident in registers), masks it, runs the fp32 online softmax in the exp2
 // domain, turns P into the B operand with movmatrix, and accumulates
 // O^T += V^T P^T with ldmatrix.trans fragments of V.  At the end of a unit
-// the warps merge through shared memory; a unit split over several CTAs
-// leaves one partial record (m, l, o) per CTA in the workspace, and the CTA
-// that takes the unit's last ticket merges them and writes bf16 out and lse.
+// the warps merge through shared memory and the CTA writes one partial
+// record (m, l, o) of the unit for the phase; the combine kernel merges the
+// records of both phases and writes bf16 out and lse.
 #include "common.cuh"
 #include "internal.h"
 
@@ -45,6 +45,10 @@ template <int D, int NB>
 struct DecCfg {
     static constexpr int kWarps = D == 256 ? 8 : 4;
     static constexpr int kThreads = 32 * kWarps;
+    // D <= 128 with up to 8 heads per group: registers for four CTAs per SM,
+    // so that three fit beside a CTA of the selection kernel when both are
+    // resident (16 heads would spill at that bound)
+    static constexpr int kMinBlocks = D == 256 ? 1 : (NB == 1 ? 4 : 3);
     static constexpr int kBufs = D == 256 ? 1 : 2;      // page buffers per warp
     static constexpr int kHalf = 32 * D;                // bytes of one page's K (or V) tile
     static constexpr int kPageBytes = 2 * kHalf;
@@ -58,7 +62,7 @@ struct DecCfg {
     static __host__ __device__ size_t smem_bytes(int units) {
         return 1024 /* alignment slack */ + kStageArea + kMl + kItems + unit_bytes(units);
     }
-    // uoff [units + 1] | uinfo [units] (int2: seq_len, n_sel | n_blo << 30 | n_bhi << 31)
+    // uoff [units + 1] | uinfo [units] (int2: validated seq_len, unused)
     static __host__ __device__ size_t unit_bytes(int units) {
         return (((size_t)(units + 1) * 4 + 15) & ~(size_t)15) + (size_t)units * 8;
     }
@@ -77,107 +81,47 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// What one unit reads, as counts of the five page groups of its work list.
-struct UnitPlan {
-    int b, g, L, Pe, We, np, c_lo, c_hi;
-    int n_pre, n_blo, n_sel, n_bhi, n_win;
-    const int32_t* sel;
-    __device__ int total() const { return n_pre + n_blo + n_sel + n_bhi + n_win; }
+// Token masks of a work item: which tokens of its page are attended.
+constexpr int kMaskAll = 0;     // every valid token (t < L)
+constexpr int kMaskFixed = 1;   // prefix or window tokens (t < Pe or t >= L - We)
+constexpr int kMaskRest = 2;    // the others (Pe <= t < L - We)
+
+// Fixed list of a unit: the pages holding prefix or window tokens, ascending:
+// [0, c_lo) | c_lo when it holds prefix tokens | c_hi - 1 when it holds
+// window tokens | [c_hi, np).  With no page left to select from (or in dense
+// mode) it is every page, unmasked.
+struct FixedList {
+    int n_pre, n_blo, n_bhi, n_win;
+    __device__ int total() const { return n_pre + n_blo + n_bhi + n_win; }
 };
 
-__device__ UnitPlan make_plan(const DecodeParams& p, int u) {
-    UnitPlan q;
-    q.b = u / p.s.Hkv;
-    q.g = u % p.s.Hkv;
-    // first round of loads together: length, selection count, first entry
-    int L = p.seq_lens[q.b];
-    const int32_t* sel_u = p.dense ? nullptr : p.sel + (size_t)u * p.s.max_sel;
-    int ns = p.dense ? 0 : p.n_sel[u];
-    const int first_raw = p.dense ? -1 : sel_u[0];
-    if (L < 0 || L > p.s.MP * kPage) {
-        latch_flag(p.flags, CSA_DEVFLAG_BAD_SEQ_LEN);
-        L = 0;
+__device__ __forceinline__ FixedList fixed_list(const SeqGeom& sg, bool dense) {
+    FixedList f;
+    f.n_blo = f.n_bhi = f.n_win = 0;
+    if (dense || sg.c_lo == sg.c_hi) {
+        f.n_pre = sg.np;
+        return f;
     }
-    const SeqGeom sg = seq_geom(L, p.prefix, p.window);
-    q.L = L;
-    q.Pe = sg.Pe;
-    q.We = sg.We;
-    q.np = sg.np;
-    q.c_lo = sg.c_lo;
-    q.c_hi = sg.c_hi;
-    q.sel = nullptr;
-    q.n_blo = q.n_sel = q.n_bhi = 0;
-    if (p.dense || sg.c_lo == sg.c_hi) {     // every valid token is attended
-        q.n_pre = sg.np;
-        q.n_win = 0;
-        return q;
-    }
-    q.n_pre = sg.c_lo;
-    q.n_win = sg.np - sg.c_hi;
-    const int cap = p.s.max_sel < sg.c_hi - sg.c_lo ? p.s.max_sel : sg.c_hi - sg.c_lo;
-    if (ns < 0 || ns > cap) {
-        latch_flag(p.flags, CSA_DEVFLAG_BAD_SELECTION);
-        ns = ns < 0 ? 0 : cap;
-    }
-    q.n_sel = ns;
-    q.sel = sel_u;
-    const int first = ns > 0 ? first_raw : -1;
-    const int last = ns > 0 ? sel_u[ns - 1] : -1;
-    const bool lo_partial = (sg.Pe % kPage) != 0;
-    const bool hi_partial = sg.We > 0 && ((L - sg.We) % kPage) != 0;
-    q.n_blo = (lo_partial && first != sg.c_lo) ? 1 : 0;
-    q.n_bhi = (hi_partial && last != sg.c_hi - 1 && !(sg.c_hi - 1 == sg.c_lo && q.n_blo)) ? 1 : 0;
-    return q;
+    f.n_pre = sg.c_lo;
+    f.n_blo = (sg.Pe % kPage) != 0 ? 1 : 0;
+    const bool hi_partial = sg.We > 0 && ((sg.L - sg.We) % kPage) != 0;
+    f.n_bhi = (hi_partial && !(sg.c_hi - 1 == sg.c_lo && f.n_blo)) ? 1 : 0;
+    f.n_win = sg.np - sg.c_hi;
+    return f;
 }
 
-// The plan of unit u again, from the (seq_len, packed counts) kept in
-// shared memory by the first pass: no global loads.
-__device__ __forceinline__ UnitPlan cached_plan(const DecodeParams& p, int u, int2 info) {
-    UnitPlan q;
-    q.b = u / p.s.Hkv;
-    q.g = u % p.s.Hkv;
-    const SeqGeom sg = seq_geom(info.x, p.prefix, p.window);
-    q.L = info.x;
-    q.Pe = sg.Pe;
-    q.We = sg.We;
-    q.np = sg.np;
-    q.c_lo = sg.c_lo;
-    q.c_hi = sg.c_hi;
-    q.n_sel = info.y & 0x3fffffff;
-    q.n_blo = (info.y >> 30) & 1;
-    q.n_bhi = (int)(((unsigned)info.y >> 31) & 1u);
-    q.sel = p.sel ? p.sel + (size_t)u * p.s.max_sel : nullptr;
-    if (p.dense || sg.c_lo == sg.c_hi) {
-        q.n_pre = sg.np;
-        q.n_win = 0;
-    } else {
-        q.n_pre = sg.c_lo;
-        q.n_win = sg.np - sg.c_hi;
-    }
-    return q;
-}
-
-// Item j of a unit's list -> logical page and whether all its valid tokens
-// are attended (else the prefix/window token mask applies).  Returns false
-// for a selection entry that is out of range or out of order.
-__device__ bool plan_item(const UnitPlan& q, int j, int& page, bool& whole) {
-    if (j < q.n_pre) { page = j; whole = true; return true; }
-    j -= q.n_pre;
-    if (j < q.n_blo) { page = q.c_lo; whole = false; return true; }
-    j -= q.n_blo;
-    if (j < q.n_sel) {
-        page = q.sel[j];
-        whole = true;
-        const bool in_range = page >= q.c_lo && page < q.c_hi;
-        const bool ordered = j == 0 || q.sel[j - 1] < page;
-        return in_range && ordered;
-    }
-    j -= q.n_sel;
-    if (j < q.n_bhi) { page = q.c_hi - 1; whole = false; return true; }
-    j -= q.n_bhi;
-    page = q.c_hi + j;
-    whole = true;
-    return true;
+__device__ __forceinline__ void fixed_item(const SeqGeom& sg, const FixedList& f, int j,
+                                           int& page, int& mask) {
+    mask = kMaskAll;
+    if (j < f.n_pre) { page = j; return; }
+    j -= f.n_pre;
+    mask = kMaskFixed;
+    if (j < f.n_blo) { page = sg.c_lo; return; }
+    j -= f.n_blo;
+    if (j < f.n_bhi) { page = sg.c_hi - 1; return; }
+    j -= f.n_bhi;
+    mask = kMaskAll;
+    page = sg.c_hi + j;
 }
 
 // Unit whose list holds flattened item x (largest u with uoff[u] <= x).
@@ -204,9 +148,11 @@ __host__ __device__ __forceinline__ size_t record_stride(int G, int D) {
     return ((size_t)G * D + 2 * G + 3) & ~(size_t)3;
 }
 
-// Combine kernel: merges the partial records of every unit split over
-// several decode CTAs, written by CTAs first .. last (rec_range):
+// Combine kernel: merges the partial records of every unit, written in phase
+// 0 (fixed pages) by CTAs rec_range.x .. .y and in phase 1 (selected pages)
+// by CTAs .z .. .w:
 //   M = max_r m_r,  out = sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r.
+// A unit without records (nothing attended) gets out = 0 and lse = -inf.
 // A CTA covers 64 float4 columns of one unit's [G][D] output; its 256 threads
 // split the records four ways (online max-rescaled sums, merged with
 // shuffles), so no thread walks all the records.
@@ -217,8 +163,7 @@ __global__ void __launch_bounds__(256) combine_kernel(DecodeParams p) {
     pdl_wait();                 // the records belong to the decode kernel
     pdl_launch_dependents();
     const int u = blockIdx.y;
-    const int2 rr = p.rec_range[u];
-    if (rr.y < rr.x) return;   // unit handled by a single CTA (or empty)
+    const int4 rr = p.rec_range[u];
     const int G = p.s.G, Hq = p.s.Hq;
     const int cols = G * D / 4;
     const int c = blockIdx.x * kCombineCols + (threadIdx.x & (kCombineCols - 1));
@@ -227,8 +172,11 @@ __global__ void __launch_bounds__(256) combine_kernel(DecodeParams p) {
     const int cc = c < cols ? c : cols - 1;
     const int h = (4 * cc) / D;
     const size_t rs = record_stride(G, D);
-    const float* base = p.partials + ((size_t)rr.x + u) * rs;
-    const int nrec = rr.y - rr.x + 1;
+    const int n0 = rr.y >= rr.x ? rr.y - rr.x + 1 : 0;
+    const int n1 = rr.w >= rr.z ? rr.w - rr.z + 1 : 0;
+    const float* base0 = p.partials + ((size_t)rr.x + u) * rs;
+    const float* base1 = p.partials + p.phase_floats + ((size_t)rr.z + u) * rs;
+    const int nrec = n0 + n1;
     float m = -INFINITY, l = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int r0 = grp; r0 < nrec; r0 += 4 * 4) {
@@ -237,7 +185,9 @@ __global__ void __launch_bounds__(256) combine_kernel(DecodeParams p) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int r = r0 + 4 * k;
-            const float* rc = base + (size_t)(r < nrec ? r : 0) * rs;
+            const float* rc = r < n0 ? base0 + (size_t)r * rs
+                                     : (r < nrec ? base1 + (size_t)(r - n0) * rs
+                                                 : (n0 > 0 ? base0 : base1));
             mr[k] = r < nrec ? __ldcg(rc + (size_t)G * D + h) : -INFINITY;
             lr[k] = __ldcg(rc + (size_t)G * D + G + h);
             v[k] = __ldcg(reinterpret_cast<const float4*>(rc) + cc);
@@ -310,7 +260,7 @@ __device__ __forceinline__ void load_page(uint32_t buf, const uint16_t* kt, cons
 }
 
 template <int D, int NB>
-__global__ void __launch_bounds__(DecCfg<D, NB>::kThreads)
+__global__ void __launch_bounds__(DecCfg<D, NB>::kThreads, DecCfg<D, NB>::kMinBlocks)
 decode_kernel(DecodeParams p) {
     using C = DecCfg<D, NB>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -327,85 +277,20 @@ decode_kernel(DecodeParams p) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Hkv = p.s.Hkv, G = p.s.G, Hq = p.s.Hq;
-    // the selection, the appended tokens and the previous users of the
-    // workspace belong to earlier kernels
-    pdl_wait();
-    pdl_launch_dependents();
-
-    // ---- per-unit list lengths and their exclusive scan
+    int2* rr2 = reinterpret_cast<int2*>(p.rec_range);   // [unit][phase]: first, last CTA
+    if (!p.early) {   // wait for everything ahead before reading anything
+        pdl_wait();
+        pdl_launch_dependents();
+    }
     for (int u = tid; u < units; u += C::kThreads) {
-        const UnitPlan q = make_plan(p, u);
-        uoff[u] = q.total();
-        uinfo[u] = make_int2(q.L, q.n_sel | (q.n_blo << 30) | (q.n_bhi << 31));
-    }
-    __syncthreads();
-    if (warp == 0) {
-        int carry = 0;
-        for (int base = 0; base < units; base += 32) {
-            const int u = base + lane;
-            const int v = u < units ? uoff[u] : 0;
-            int incl = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            if (u < units) uoff[u] = carry + incl - v;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
+        int L = p.seq_lens[u / Hkv];
+        if (L < 0 || L > p.s.MP * kPage) {
+            latch_flag(p.flags, CSA_DEVFLAG_BAD_SEQ_LEN);
+            L = 0;
         }
-        if (lane == 0) uoff[units] = carry;
+        uinfo[u] = make_int2(L, 0);
     }
-    __syncthreads();
-    const long long T = uoff[units];
-    // partition over at most T CTAs so that every participating CTA owns at
-    // least one item: the merge counts every CTA between a unit's first and
-    // last one
-    // at least kMinItems pages per CTA: fewer partial records per unit to
-    // merge when the attended set is small
-    constexpr long long kMinItems = 4 * C::kWarps;
-    long long want = (T + kMinItems - 1) / kMinItems;
-    if (want < 1) want = 1;
-    const int n_cta = (int)(want < (long long)gridDim.x ? want : gridDim.x);
-    const long long s = blockIdx.x < (unsigned)n_cta ? T * blockIdx.x / n_cta : T;
-    const long long e = blockIdx.x < (unsigned)n_cta ? T * (blockIdx.x + 1) / n_cta : T;
 
-    // units with nothing to attend (empty sequences): out = 0, lse = -inf
-    if (blockIdx.x == 0) {
-        for (int u = 0; u < units; ++u) {
-            if (uoff[u + 1] != uoff[u]) continue;
-            if (tid == 0) p.rec_range[u] = make_int2(0, -1);
-            const int b = u / Hkv, g = u % Hkv;
-            for (int i = tid; i < G * D; i += C::kThreads) {
-                const int h = i / D, c = i % D;
-                p.out[((size_t)b * Hq + (size_t)g * G + h) * D + c] = 0;
-                if (c == 0 && p.lse) p.lse[(size_t)b * Hq + (size_t)g * G + h] = -INFINITY;
-            }
-        }
-    }
-    if (s >= e) return;
-
-    // ---- resolve the physical page of every item of this CTA's slice
-    for (long long x = s + tid; x < e; x += C::kThreads) {
-        const int u = find_unit(uoff, units, x);
-        const UnitPlan q = cached_plan(p, u, uinfo[u]);
-        int page = 0;
-        bool whole = true;
-        int phys = -1;
-        if (!plan_item(q, (int)(x - uoff[u]), page, whole)) {
-            latch_flag(p.flags, CSA_DEVFLAG_BAD_SELECTION);
-        } else {
-            phys = p.page_table[(size_t)q.b * p.s.MP + page];
-            if (phys < 0 || phys >= p.s.NPG) {
-                latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
-                phys = -1;
-            }
-        }
-        items[x - s] = make_int2(phys, page * 2 + (whole ? 1 : 0));
-    }
-    __syncthreads();
-
-    const int u_first = find_unit(uoff, units, s);
-    const int u_last = find_unit(uoff, units, e - 1);
     const int gq = lane >> 2, tq = lane & 3;
     const int mi = lane >> 3, ri = lane & 7;
     // per-lane ldmatrix geometry (chunk c of row r sits at c ^ (r & 7))
@@ -413,214 +298,297 @@ decode_kernel(DecodeParams p) {
     const int v_tok = ri + ((mi >> 1) << 3), v_half = mi & 1;
     const float sl2 = p.scale_log2;
     const uint32_t wbuf = smem_u32(stages) + (uint32_t)(warp * C::kBufs * C::kPageBytes);
+    const size_t rs = record_stride(G, D);
 
-    for (int u = u_first; u <= u_last; ++u) {
-        const long long a = s > uoff[u] ? s : uoff[u];
-        const long long bnd = e < uoff[u + 1] ? e : uoff[u + 1];
-        if (a >= bnd) continue;
-        const int b = u / Hkv, g = u % Hkv;
-        const int L = uinfo[u].x;
-        const SeqGeom sg = seq_geom(L, p.prefix, p.window);
-        const int Pe = sg.Pe, Lw = L - sg.We;
-
-        // Q^T as the B operand: b0 = q[head][16kb + 2tq, +1], b1 = +8
-        uint32_t qf[C::kMB][NB][2];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-            const int head = nb * 8 + gq;
-            const uint32_t* qw = reinterpret_cast<const uint32_t*>(
-                p.q + ((size_t)b * Hq + (size_t)g * G + (head < G ? head : 0)) * D);
-#pragma unroll
-            for (int kb = 0; kb < C::kMB; ++kb) {
-                qf[kb][nb][0] = head < G ? __ldg(qw + 8 * kb + tq) : 0u;
-                qf[kb][nb][1] = head < G ? __ldg(qw + 8 * kb + 4 + tq) : 0u;
-            }
+    // Phase 0 streams the fixed pages (prefix and window), which do not depend
+    // on the selection; phase 1 the selected pages.  With p.early set, phase 0
+    // runs while the selection kernel ahead is still working.
+    for (int ph = 0; ph < 2; ++ph) {
+        if (ph == 1 && p.early) {
+            pdl_wait();         // the selection is complete and visible
+            pdl_launch_dependents();
         }
-        float m[NB][2], l[NB][2], o[C::kMB][NB][4];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-            m[nb][0] = m[nb][1] = -INFINITY;
-            l[nb][0] = l[nb][1] = 0.f;
-#pragma unroll
-            for (int mb = 0; mb < C::kMB; ++mb)
-                o[mb][nb][0] = o[mb][nb][1] = o[mb][nb][2] = o[mb][nb][3] = 0.f;
-        }
-
-        // this warp's items of the segment: a + warp, a + warp + kWarps, ...
-        auto issue = [&](long long x, int slot) {
-            const int2 it = items[x - s];
-            if (it.x >= 0) {
-                const int page = it.y >> 1;
-                const size_t tile = ((size_t)it.x * Hkv + g) * kPage * D;
-                const int rows = L - page * kPage < kPage ? L - page * kPage : kPage;
-                load_page<D>(wbuf + (uint32_t)(slot * C::kPageBytes), p.k_cache + tile,
-                             p.v_cache + tile, rows, lane);
+        __syncthreads();        // uinfo written; smem of the previous phase free
+        // ---- per-unit list lengths and their exclusive scan
+        for (int u = tid; u < units; u += C::kThreads) {
+            const SeqGeom sg = seq_geom(uinfo[u].x, p.prefix, p.window);
+            int n = 0;
+            if (ph == 0) {
+                n = fixed_list(sg, p.dense).total();
+            } else if (!p.dense && sg.c_lo < sg.c_hi) {
+                n = p.n_sel[u];
+                const int cap = p.s.max_sel < sg.c_hi - sg.c_lo ? p.s.max_sel : sg.c_hi - sg.c_lo;
+                if (n < 0 || n > cap) {
+                    latch_flag(p.flags, CSA_DEVFLAG_BAD_SELECTION);
+                    n = n < 0 ? 0 : cap;
+                }
             }
-            cp_async_commit();
-        };
-        long long x = a + warp;
-        int slot = 0;
-        if (x < bnd) issue(x, 0);
-        for (; x < bnd; x += C::kWarps) {
-            const long long xn = x + C::kWarps;
-            if (C::kBufs == 2) {
-                if (xn < bnd) {
-                    issue(xn, slot ^ 1);
-                    cp_async_wait<1>();
+            uoff[u] = n;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int carry = 0;
+            for (int base = 0; base < units; base += 32) {
+                const int u = base + lane;
+                const int v = u < units ? uoff[u] : 0;
+                int incl = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                if (u < units) uoff[u] = carry + incl - v;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) uoff[units] = carry;
+        }
+        __syncthreads();
+        const long long T = uoff[units];
+        // at least kMinItems pages per CTA (fewer partial records to merge;
+        // measured faster than one or two pages per warp in either phase),
+        // and every participating CTA owns at least one item
+        constexpr long long kMinItems = 4 * C::kWarps;
+        long long want = (T + kMinItems - 1) / kMinItems;
+        if (want < 1) want = 1;
+        const int n_cta = (int)(want < (long long)gridDim.x ? want : gridDim.x);
+        const long long s = blockIdx.x < (unsigned)n_cta ? T * blockIdx.x / n_cta : T;
+        const long long e = blockIdx.x < (unsigned)n_cta ? T * (blockIdx.x + 1) / n_cta : T;
+        if (blockIdx.x == 0) {   // units without pages in this phase: no records
+            for (int u = tid; u < units; u += C::kThreads)
+                if (uoff[u + 1] == uoff[u]) rr2[2 * u + ph] = make_int2(0, -1);
+        }
+        if (s >= e) continue;
+
+        // ---- resolve the physical page of every item of this CTA's slice
+        for (long long x = s + tid; x < e; x += C::kThreads) {
+            const int u = find_unit(uoff, units, x);
+            const int b = u / Hkv;
+            const int j = (int)(x - uoff[u]);
+            const SeqGeom sg = seq_geom(uinfo[u].x, p.prefix, p.window);
+            int page = 0, mask = kMaskAll;
+            bool ok = true;
+            if (ph == 0) {
+                fixed_item(sg, fixed_list(sg, p.dense), j, page, mask);
+            } else {
+                const int32_t* su = p.sel + (size_t)u * p.s.max_sel;
+                page = su[j];
+                mask = kMaskRest;
+                ok = page >= sg.c_lo && page < sg.c_hi && (j == 0 || su[j - 1] < page);
+                if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_SELECTION);
+            }
+            int phys = -1;
+            if (ok) {
+                phys = p.page_table[(size_t)b * p.s.MP + page];
+                if (phys < 0 || phys >= p.s.NPG) {
+                    latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
+                    phys = -1;
+                }
+            }
+            items[x - s] = make_int2(phys, page * 4 + mask);
+        }
+        __syncthreads();
+
+        const int u_first = find_unit(uoff, units, s);
+        const int u_last = find_unit(uoff, units, e - 1);
+        float* region = p.partials + (size_t)ph * p.phase_floats;
+
+        for (int u = u_first; u <= u_last; ++u) {
+            const long long a = s > uoff[u] ? s : uoff[u];
+            const long long bnd = e < uoff[u + 1] ? e : uoff[u + 1];
+            if (a >= bnd) continue;
+            const int b = u / Hkv, g = u % Hkv;
+            const int L = uinfo[u].x;
+            const SeqGeom sg = seq_geom(L, p.prefix, p.window);
+            const int Pe = sg.Pe, Lw = L - sg.We;
+
+            // Q^T as the B operand: b0 = q[head][16kb + 2tq, +1], b1 = +8
+            uint32_t qf[C::kMB][NB][2];
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int head = nb * 8 + gq;
+                const uint32_t* qw = reinterpret_cast<const uint32_t*>(
+                    p.q + ((size_t)b * Hq + (size_t)g * G + (head < G ? head : 0)) * D);
+#pragma unroll
+                for (int kb = 0; kb < C::kMB; ++kb) {
+                    qf[kb][nb][0] = head < G ? __ldg(qw + 8 * kb + tq) : 0u;
+                    qf[kb][nb][1] = head < G ? __ldg(qw + 8 * kb + 4 + tq) : 0u;
+                }
+            }
+            float m[NB][2], l[NB][2], o[C::kMB][NB][4];
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                m[nb][0] = m[nb][1] = -INFINITY;
+                l[nb][0] = l[nb][1] = 0.f;
+#pragma unroll
+                for (int mb = 0; mb < C::kMB; ++mb)
+                    o[mb][nb][0] = o[mb][nb][1] = o[mb][nb][2] = o[mb][nb][3] = 0.f;
+            }
+
+            // this warp's items of the segment: a + warp, a + warp + kWarps, ...
+            auto issue = [&](long long x, int slot) {
+                const int2 it = items[x - s];
+                if (it.x >= 0) {
+                    const int page = it.y >> 2;
+                    const size_t tile = ((size_t)it.x * Hkv + g) * kPage * D;
+                    const int rows = L - page * kPage < kPage ? L - page * kPage : kPage;
+                    load_page<D>(wbuf + (uint32_t)(slot * C::kPageBytes), p.k_cache + tile,
+                                 p.v_cache + tile, rows, lane);
+                }
+                cp_async_commit();
+            };
+            long long x = a + warp;
+            int slot = 0;
+            if (x < bnd) issue(x, 0);
+            for (; x < bnd; x += C::kWarps) {
+                const long long xn = x + C::kWarps;
+                if (C::kBufs == 2) {
+                    if (xn < bnd) {
+                        issue(xn, slot ^ 1);
+                        cp_async_wait<1>();
+                    } else {
+                        cp_async_wait<0>();
+                    }
                 } else {
                     cp_async_wait<0>();
                 }
-            } else {
-                cp_async_wait<0>();
-            }
-            __syncwarp();
-            const int2 it = items[x - s];
-            if (it.x >= 0) {
-                const int page = it.y >> 1;
-                const bool whole = it.y & 1;
-                const uint32_t kbase = wbuf + (uint32_t)(slot * C::kPageBytes);
-                const uint32_t vbase = kbase + C::kHalf;
-                // ---- S^T = K Q^T
-                float sacc[NB][4];
-#pragma unroll
-                for (int nb = 0; nb < NB; ++nb)
-                    sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
-#pragma unroll
-                for (int kb = 0; kb < C::kMB; ++kb) {
-                    const int chunk = 2 * kb + k_half;
-                    const uint32_t addr = kbase + (chunk >> 3) * 2048 + k_tok * 128 +
-                                          (((chunk & 7) ^ ri) << 4);
-                    uint32_t af[4];
-                    ldsm_x4(af, addr);
+                __syncwarp();
+                const int2 it = items[x - s];
+                if (it.x >= 0) {
+                    const int page = it.y >> 2;
+                    const int mask = it.y & 3;
+                    const uint32_t kbase = wbuf + (uint32_t)(slot * C::kPageBytes);
+                    const uint32_t vbase = kbase + C::kHalf;
+                    // ---- S^T = K Q^T
+                    float sacc[NB][4];
 #pragma unroll
                     for (int nb = 0; nb < NB; ++nb)
-                        mma_bf16_16816(sacc[nb], af, qf[kb][nb][0], qf[kb][nb][1]);
-                }
-                // ---- mask and online softmax (exp2 domain)
-                const int t0 = page * kPage + gq, t1 = t0 + 8;
-                const bool in0 = t0 < L && (whole || t0 < Pe || t0 >= Lw);
-                const bool in1 = t1 < L && (whole || t1 < Pe || t1 >= Lw);
-                uint32_t pb[NB][2];
+                        sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    const float s00 = in0 ? sacc[nb][0] * sl2 : -INFINITY;
-                    const float s01 = in0 ? sacc[nb][1] * sl2 : -INFINITY;
-                    const float s10 = in1 ? sacc[nb][2] * sl2 : -INFINITY;
-                    const float s11 = in1 ? sacc[nb][3] * sl2 : -INFINITY;
-                    float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+                    for (int kb = 0; kb < C::kMB; ++kb) {
+                        const int chunk = 2 * kb + k_half;
+                        const uint32_t addr = kbase + (chunk >> 3) * 2048 + k_tok * 128 +
+                                              (((chunk & 7) ^ ri) << 4);
+                        uint32_t af[4];
+                        ldsm_x4(af, addr);
 #pragma unroll
-                    for (int o2 = 4; o2 < 32; o2 <<= 1) {
-                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
-                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+                        for (int nb = 0; nb < NB; ++nb)
+                            mma_bf16_16816(sacc[nb], af, qf[kb][nb][0], qf[kb][nb][1]);
                     }
-                    const float mn0 = fmaxf(m[nb][0], mx0), mn1 = fmaxf(m[nb][1], mx1);
-                    const float base0 = mn0 == -INFINITY ? 0.f : mn0;
-                    const float base1 = mn1 == -INFINITY ? 0.f : mn1;
-                    const float al0 = ex2(m[nb][0] - base0), al1 = ex2(m[nb][1] - base1);
-                    const uint32_t P0 = pack_bf16x2(ex2(s00 - base0), ex2(s01 - base1));
-                    const uint32_t P1 = pack_bf16x2(ex2(s10 - base0), ex2(s11 - base1));
-                    l[nb][0] = l[nb][0] * al0 + bf16_lo(P0) + bf16_lo(P1);
-                    l[nb][1] = l[nb][1] * al1 + bf16_hi(P0) + bf16_hi(P1);
-                    m[nb][0] = mn0;
-                    m[nb][1] = mn1;
+                    // ---- mask and online softmax (exp2 domain)
+                    const int t0 = page * kPage + gq, t1 = t0 + 8;
+                    const bool f0 = t0 < Pe || t0 >= Lw, f1 = t1 < Pe || t1 >= Lw;
+                    const bool in0 = t0 < L && (mask == kMaskAll || (mask == kMaskFixed) == f0);
+                    const bool in1 = t1 < L && (mask == kMaskAll || (mask == kMaskFixed) == f1);
+                    uint32_t pb[NB][2];
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) {
+                        const float s00 = in0 ? sacc[nb][0] * sl2 : -INFINITY;
+                        const float s01 = in0 ? sacc[nb][1] * sl2 : -INFINITY;
+                        const float s10 = in1 ? sacc[nb][2] * sl2 : -INFINITY;
+                        const float s11 = in1 ? sacc[nb][3] * sl2 : -INFINITY;
+                        float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+#pragma unroll
+                        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+                            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+                        }
+                        const float mn0 = fmaxf(m[nb][0], mx0), mn1 = fmaxf(m[nb][1], mx1);
+                        const float base0 = mn0 == -INFINITY ? 0.f : mn0;
+                        const float base1 = mn1 == -INFINITY ? 0.f : mn1;
+                        const float al0 = ex2(m[nb][0] - base0), al1 = ex2(m[nb][1] - base1);
+                        const uint32_t P0 = pack_bf16x2(ex2(s00 - base0), ex2(s01 - base1));
+                        const uint32_t P1 = pack_bf16x2(ex2(s10 - base0), ex2(s11 - base1));
+                        l[nb][0] = l[nb][0] * al0 + bf16_lo(P0) + bf16_lo(P1);
+                        l[nb][1] = l[nb][1] * al1 + bf16_hi(P0) + bf16_hi(P1);
+                        m[nb][0] = mn0;
+                        m[nb][1] = mn1;
+#pragma unroll
+                        for (int mb = 0; mb < C::kMB; ++mb) {
+                            o[mb][nb][0] *= al0;
+                            o[mb][nb][1] *= al1;
+                            o[mb][nb][2] *= al0;
+                            o[mb][nb][3] *= al1;
+                        }
+                        pb[nb][0] = movmatrix_trans(P0);
+                        pb[nb][1] = movmatrix_trans(P1);
+                    }
+                    // ---- O^T += V^T P^T
 #pragma unroll
                     for (int mb = 0; mb < C::kMB; ++mb) {
-                        o[mb][nb][0] *= al0;
-                        o[mb][nb][1] *= al1;
-                        o[mb][nb][2] *= al0;
-                        o[mb][nb][3] *= al1;
+                        const int chunk = 2 * mb + v_half;
+                        const uint32_t addr = vbase + (chunk >> 3) * 2048 + v_tok * 128 +
+                                              (((chunk & 7) ^ ri) << 4);
+                        uint32_t af[4];
+                        ldsm_x4_trans(af, addr);
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb)
+                            mma_bf16_16816(o[mb][nb], af, pb[nb][0], pb[nb][1]);
                     }
-                    pb[nb][0] = movmatrix_trans(P0);
-                    pb[nb][1] = movmatrix_trans(P1);
                 }
-                // ---- O^T += V^T P^T
+                __syncwarp();                 // the buffer is refilled next
+                if (C::kBufs == 1) {
+                    if (xn < bnd) issue(xn, 0);
+                } else {
+                    slot ^= 1;
+                }
+            }
+
+            // ---- merge the warps of this CTA (Ow aliases the page buffers)
+            __syncthreads();
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v = l[nb][hh];
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    v += __shfl_xor_sync(0xffffffffu, v, 8);
+                    v += __shfl_xor_sync(0xffffffffu, v, 16);
+                    l[nb][hh] = v;
+                }
+                if (gq == 0) {
+                    ms[warp * C::kHeads + nb * 8 + 2 * tq] = m[nb][0];
+                    ms[warp * C::kHeads + nb * 8 + 2 * tq + 1] = m[nb][1];
+                    ls[warp * C::kHeads + nb * 8 + 2 * tq] = l[nb][0];
+                    ls[warp * C::kHeads + nb * 8 + 2 * tq + 1] = l[nb][1];
+                }
 #pragma unroll
                 for (int mb = 0; mb < C::kMB; ++mb) {
-                    const int chunk = 2 * mb + v_half;
-                    const uint32_t addr = vbase + (chunk >> 3) * 2048 + v_tok * 128 +
-                                          (((chunk & 7) ^ ri) << 4);
-                    uint32_t af[4];
-                    ldsm_x4_trans(af, addr);
-#pragma unroll
-                    for (int nb = 0; nb < NB; ++nb)
-                        mma_bf16_16816(o[mb][nb], af, pb[nb][0], pb[nb][1]);
+                    float* ow = Ow + (size_t)warp * C::kHeads * D;
+                    const int h0 = nb * 8 + 2 * tq, c0 = mb * 16 + gq;
+                    ow[(size_t)h0 * D + c0] = o[mb][nb][0];
+                    ow[(size_t)(h0 + 1) * D + c0] = o[mb][nb][1];
+                    ow[(size_t)h0 * D + c0 + 8] = o[mb][nb][2];
+                    ow[(size_t)(h0 + 1) * D + c0 + 8] = o[mb][nb][3];
                 }
             }
-            __syncwarp();                 // the buffer is refilled next
-            if (C::kBufs == 1) {
-                if (xn < bnd) issue(xn, 0);
-            } else {
-                slot ^= 1;
-            }
-        }
+            __syncthreads();
 
-        // ---- merge the warps of this CTA (Ow aliases the page buffers)
-        __syncthreads();
+            // ---- this CTA's partial record of the unit (merged by the combine kernel)
+            float* rec = region + ((size_t)blockIdx.x + u) * rs;
+            for (int idx = tid; idx < G * D; idx += C::kThreads) {
+                const int h = idx / D, c = idx % D;
+                float M = -INFINITY;
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
+                for (int w = 0; w < C::kWarps; ++w) M = fmaxf(M, ms[w * C::kHeads + h]);
+                float acc = 0.f, lsum = 0.f;
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float v = l[nb][hh];
-                v += __shfl_xor_sync(0xffffffffu, v, 4);
-                v += __shfl_xor_sync(0xffffffffu, v, 8);
-                v += __shfl_xor_sync(0xffffffffu, v, 16);
-                l[nb][hh] = v;
-            }
-            if (gq == 0) {
-                ms[warp * C::kHeads + nb * 8 + 2 * tq] = m[nb][0];
-                ms[warp * C::kHeads + nb * 8 + 2 * tq + 1] = m[nb][1];
-                ls[warp * C::kHeads + nb * 8 + 2 * tq] = l[nb][0];
-                ls[warp * C::kHeads + nb * 8 + 2 * tq + 1] = l[nb][1];
-            }
-#pragma unroll
-            for (int mb = 0; mb < C::kMB; ++mb) {
-                float* ow = Ow + (size_t)warp * C::kHeads * D;
-                const int h0 = nb * 8 + 2 * tq, c0 = mb * 16 + gq;
-                ow[(size_t)h0 * D + c0] = o[mb][nb][0];
-                ow[(size_t)(h0 + 1) * D + c0] = o[mb][nb][1];
-                ow[(size_t)h0 * D + c0 + 8] = o[mb][nb][2];
-                ow[(size_t)(h0 + 1) * D + c0 + 8] = o[mb][nb][3];
-            }
-        }
-        __syncthreads();
-
-        const int first_cta = cta_of(uoff[u], T, n_cta);
-        const int last_cta = cta_of(uoff[u + 1] - 1, T, n_cta);
-        const bool alone = first_cta == last_cta;
-        if (alone && tid == 0) p.rec_range[u] = make_int2(0, -1);   // nothing to combine
-        const size_t rs = record_stride(G, D);
-        float* rec = p.partials + ((size_t)blockIdx.x + u) * rs;
-        for (int idx = tid; idx < G * D; idx += C::kThreads) {
-            const int h = idx / D, c = idx % D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < C::kWarps; ++w) M = fmaxf(M, ms[w * C::kHeads + h]);
-            float acc = 0.f, lsum = 0.f;
-#pragma unroll
-            for (int w = 0; w < C::kWarps; ++w) {
-                const float mw = ms[w * C::kHeads + h];
-                const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
-                acc += Ow[((size_t)w * C::kHeads + h) * D + c] * f;
-                lsum += ls[w * C::kHeads + h] * f;
-            }
-            const size_t oi = ((size_t)b * Hq + (size_t)g * G + h);
-            if (alone) {
-                const float val = lsum > 0.f ? acc / lsum : 0.f;
-                p.out[oi * D + c] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
-                if (c == 0 && p.lse)
-                    p.lse[oi] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f
-                                           : -INFINITY;
-            } else {
+                for (int w = 0; w < C::kWarps; ++w) {
+                    const float mw = ms[w * C::kHeads + h];
+                    const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
+                    acc += Ow[((size_t)w * C::kHeads + h) * D + c] * f;
+                    lsum += ls[w * C::kHeads + h] * f;
+                }
                 rec[(size_t)h * D + c] = acc;
                 if (c == 0) {
                     rec[(size_t)G * D + h] = M;
                     rec[(size_t)G * D + G + h] = lsum;
                 }
             }
+            const int first_cta = cta_of(uoff[u], T, n_cta);
+            if (blockIdx.x == first_cta && tid == 0)
+                rr2[2 * u + ph] = make_int2(first_cta, cta_of(uoff[u + 1] - 1, T, n_cta));
+            __syncthreads();   // Ow / ms / ls and the page buffers are reused next
         }
-        if (!alone && blockIdx.x == first_cta && tid == 0)
-            p.rec_range[u] = make_int2(first_cta, last_cta);   // read by the combine kernel
-        __syncthreads();   // Ow / ms / ls and the page buffers are reused by the next unit
     }
 }
 

@@ -2,7 +2,6 @@
 // kernel translation units.  Not installed; the public ABI is include/csa.h.
 #pragma once
 
-#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -12,11 +11,10 @@ namespace csa {
 // Workspace layout (byte offsets into the caller's workspace).
 struct WsLayout {
     size_t flags;          // uint32 device flag word
-    size_t score_tickets;  // uint32 [units]
-    size_t rec_range;      // int2 [units]
+    size_t rec_range;      // int4 [units]
     size_t scores;         // fp32 [B][Hkv][max_pages]
-    size_t partials;       // fp32 [dec_slots][decode_record_floats]
-    size_t dec_slots;      // partial records available
+    size_t partials;       // fp32 [2][dec_slots][decode_record_floats]
+    size_t dec_slots;      // partial records available per decode phase
     size_t total;
 };
 
@@ -81,11 +79,22 @@ struct DecodeParams {
     uint16_t* out;
     float* lse;             // nullable
     uint32_t* flags;
-    int2* rec_range;        // [units]: CTAs whose partial records the combine merges
-    float* partials;        // [dec_slots][record]: o[G][D] | m[G] | l[G]
+    int4* rec_range;        // [units]: first/last CTA with a record, per phase (x,y | z,w)
+    float* partials;        // [2][dec_slots][record]: o[G][D] | m[G] | l[G]
+    size_t phase_floats;    // floats of one phase's record region (dec_slots * record)
+    int early;              // 1: the prefix/window phase runs before the dependency wait
     Shape s;
 };
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st);
+
+// Kind of the last kernel-launching call issued on a stream (host side).
+// csa_decode streams the prefix/window pages before the dependency wait only
+// when the call before it on the stream was csa_score_select: its kernels
+// wait in a chain, so every earlier kernel on the stream (the appends of
+// csa_meta_update, the previous decode's combine) has finished by then.
+enum CallKind { kCallOther = 0, kCallScoreSelect = 1 };
+void note_stream_call(const void* stream, CallKind kind);
+CallKind last_stream_call(const void* stream);
 
 // Grid sizes (shared by the workspace sizing and the launches).
 int device_sm_count();

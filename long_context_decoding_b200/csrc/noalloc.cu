@@ -92,12 +92,13 @@ extern "C" int csa_decode_noalloc(const csa_dims* d, const void* q, const void* 
     s.NPG = d->num_pages;
     s.max_sel = d->max_sel;
 
-    // scratch: [flag word | record ranges | partial records], each 256-byte aligned
+    // scratch: [flag word | record ranges | partial records of the two
+    // decode phases], each 256-byte aligned
     const size_t units = (size_t)s.B * s.Hkv;
     const size_t ranges_off = 256;
-    const size_t partials_off = ranges_off + up256(8 * units);
+    const size_t partials_off = ranges_off + up256(16 * units);
     const size_t slots = (size_t)decode_grid(s) + units;
-    const size_t need = partials_off + 4 * slots * decode_record_floats(s);
+    const size_t need = partials_off + 2 * 4 * slots * decode_record_floats(s);
     if (need > kNoAllocScratchBytes) return CSA_ERR_WORKSPACE;   // shape needs more scratch
 
     int dev = 0;
@@ -129,9 +130,12 @@ extern "C" int csa_decode_noalloc(const csa_dims* d, const void* q, const void* 
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
     p.flags = reinterpret_cast<uint32_t*>(scratch);
-    p.rec_range = reinterpret_cast<int2*>(scratch + ranges_off);
+    p.rec_range = reinterpret_cast<int4*>(scratch + ranges_off);
     p.partials = reinterpret_cast<float*>(scratch + partials_off);
+    p.phase_floats = slots * decode_record_floats(s);
+    p.early = 0;                 // the scratch is shared: wait before touching it
     p.s = s;
+    note_stream_call(stream, kCallOther);
     if (launch_decode(p, st) != cudaSuccess) {
         cudaGetLastError();
         return CSA_ERR_CUDA;

@@ -213,3 +213,19 @@ def test_repeat_calls_reuse_workspace(cuda):
         out2, _ = run.gpu_decode(run.layer.sel, run.layer.n_sel)
     torch.cuda.synchronize()
     assert torch.equal(out1, out2)
+
+
+def test_fixed_pages_streamed_before_the_selection_ends(cuda):
+    """Right after csa_score_select on the same stream, the decode streams the
+    prefix and window pages while the selection kernel still runs; the result
+    is bit-identical to a decode that waits for everything first."""
+    run = Run(wl.make_case(wl.CTX32K, cuda))
+    run.gpu_meta()
+    for _ in range(3):
+        run.gpu_select(scores=False)
+        out_e, lse_e = run.gpu_decode(run.layer.sel, run.layer.n_sel)   # overlapped
+        out_w, lse_w = run.gpu_decode(run.layer.sel, run.layer.n_sel)   # waits first
+        torch.cuda.synchronize()
+        assert torch.equal(out_e, out_w)
+        assert torch.equal(lse_e, lse_w)
+    assert csa.device_status(run.ws) == 0
