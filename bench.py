@@ -5,13 +5,14 @@
                     [--workload ctx256k|ctx64k]
 
 One step = one decode step of the whole hot path for every layer of the
-workload: append the new token + metadata update, Quest scoring + top-k
-selection, split-K sparse decode + merge.  The default workload is the
+workload: append the new token + metadata update (csa_meta_update), then
+Quest scoring, top-k selection and the split-K sparse decode + merge in one
+csa_sparse_attention call.  The default workload is the
 12-layer, batch-4, 262144-token stack (32 query / 4 kv heads, head dim 128,
 prefix 128, per-layer (window, budget) cycling through (512, 1024) ...
 (4096, 8192)); its inputs are synthetic (seeded Gaussian q/K/V in a paged
 cache with a random page permutation).  Each step is one CUDA graph of the
-36 library calls; the K timed steps are replayed back to back between CUDA
+24 library calls; the K timed steps are replayed back to back between CUDA
 events.  Every layer touches 150-235 MB (1.8-2.8 GB per step), more than the
 126 MB L2, so no flush is needed between steps.
 
@@ -272,19 +273,24 @@ class Stack:
             if what in ("all",):
                 csa.meta_update(self.d, lay.k_cache, lay.v_cache, lay.meta, lay.page_table, lens,
                                 nk_, nv_, 1, self.ws)
-            if what in ("all", "select"):
+            if what in ("all", "sparse"):
+                csa.sparse_attention(self.d, q_, lay.k_cache, lay.v_cache, lay.meta,
+                                     lay.page_table, lens, lay.prefix, lay.window, lay.budget,
+                                     lay.sel, lay.n_sel, lay.out, self.ws, lay.lse)
+            if what in ("select",):
                 csa.score_select(self.d, q_, lay.meta, lay.page_table, lens, lay.prefix,
                                  lay.window, lay.budget, lay.sel, lay.n_sel, self.ws)
-            if what in ("all", "decode"):
+            if what in ("decode",):
                 csa.decode(self.d, q_, lay.k_cache, lay.v_cache, lay.page_table, lens, lay.sel,
                            lay.n_sel, lay.prefix, lay.window, lay.out, self.ws, lay.lse)
 
     def launches_per_step(self) -> int:
-        """Kernels of one step: per layer meta update, score (only when pages
-        are selected), select, decode and its split-K combine."""
+        """Kernels of one step: per layer the metadata update, then the scoring
+        kernel, the fused selection + decode kernel and the split-K combine
+        (or, with nothing to select, the selection, decode and combine)."""
         n = 0
         for lay in self.layers:
-            n += 1 + (1 if lay.budget // 16 > 0 else 0) + 1 + 2
+            n += 1 + 3
         return n
 
     def graph(self, fn):
@@ -382,6 +388,7 @@ def run_ours(args, dist: Dist, base: wl.Workload):
         # the scoring kernel over every candidate, followed by a selection
         # kernel that has nothing to select.
         s_last = W + K - 1
+        g_spa = st.graph(lambda: st.calls(s_last, what="sparse"))
         g_sel = st.graph(lambda: st.calls(s_last, what="select"))
         g_dec = st.graph(lambda: st.calls(s_last, what="decode"))
         sc_buf = torch.empty((w.B, w.Hkv, w.max_pages), dtype=torch.float32, device=dev)
@@ -395,7 +402,8 @@ def run_ours(args, dist: Dist, base: wl.Workload):
         g_sco = st.graph(score_only)
         reps = 5
         times = {}
-        for name, g in (("score", g_sco), ("score_select", g_sel), ("decode", g_dec)):
+        for name, g in (("score", g_sco), ("sparse_attention", g_spa), ("score_select", g_sel),
+                        ("decode", g_dec)):
             time_graphs([g])
             times[name] = time_graphs([g], reps) / (reps * nl)
         bl = st.bytes_per_layer(s_last)
@@ -403,6 +411,10 @@ def run_ours(args, dist: Dist, base: wl.Workload):
         dec_bytes = sum(x["kv"] + x["q_out"] for x in bl) / nl
         calls = {"score": {"us": 1e6 * times["score"], "bytes": meta_bytes,
                            "gbs": meta_bytes / times["score"] / 1e9},
+                 "sparse_attention": {"us": 1e6 * times["sparse_attention"],
+                                      "bytes": meta_bytes + dec_bytes,
+                                      "gbs": (meta_bytes + dec_bytes) / times["sparse_attention"]
+                                      / 1e9},
                  "score_select": {"us": 1e6 * times["score_select"], "bytes": meta_bytes,
                                   "gbs": meta_bytes / times["score_select"] / 1e9},
                  "decode": {"us": 1e6 * times["decode"], "bytes": dec_bytes,
@@ -442,7 +454,7 @@ def run_ours(args, dist: Dist, base: wl.Workload):
 
 def e2e(st: Stack, K: int, W: int, dist: Dist):
     """Per step: H2D copy of the step's q/new_k/new_v (pinned host memory),
-    the 36 library calls, D2H copy of every layer's output; one CUDA graph
+    the 24 library calls, D2H copy of every layer's output; one CUDA graph
     per step, K steps timed."""
     nl = len(st.layers)
     host_in, dev_in, host_out = [], [], []
@@ -472,14 +484,13 @@ def e2e(st: Stack, K: int, W: int, dist: Dist):
     d2h = sum(t_.numel() * t_.element_size() for t_ in host_out[0])
     return {"value": dist.world * st.w.B * nl * K / t, "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
-            "path": "pinned host -> device copies, csa_meta_update / csa_score_select / "
-                    "csa_decode per layer, device -> pinned host copy of out; one CUDA graph "
-                    "per step"}
+            "path": "pinned host -> device copies, csa_meta_update / csa_sparse_attention "
+                    "per layer, device -> pinned host copy of out; one CUDA graph per step"}
 
 
 def secondary_64k(dev, dist: Dist):
-    """The 64k single-layer workload: one layer step (score + select +
-    decode, no append) per graph; a 256 MB read between replays flushes L2
+    """The 64k single-layer workload: one layer step (one
+    csa_sparse_attention call: score, select, decode; no append) per graph; a 256 MB read between replays flushes L2
     (the layer itself moves only ~84 MB).  The flush reads rather than
     writes, so that no dirty L2 lines are written back during the timed
     replay."""
@@ -493,7 +504,7 @@ def secondary_64k(dev, dist: Dist):
     scrub = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MB
 
     def body():
-        lay.step(c.q)
+        lay.step(c.q, fused=True)
 
     body()
     torch.cuda.synchronize()

@@ -199,6 +199,23 @@ int csa_decode_full(const csa_dims *d, const void *q, const void *k_cache,
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * One call for the sparse part of a decode step: the Quest scoring and
+ * top-k selection of csa_score_select followed by the attention of
+ * csa_decode over the pages it selected (same arguments, meanings and
+ * outputs: sel_pages and n_sel receive the selection, out and lse the
+ * attention).  Up to 32 (sequence, kv-head) units with at least one page to
+ * select run the selection and the decode of the selected pages in one
+ * launch, the prefix and window pages being decoded meanwhile by other CTAs
+ * of the same grid; other shapes run the separate kernels.  Reads
+ * `page_table` and `seq_lens` early, like csa_score_select.
+ */
+int csa_sparse_attention(const csa_dims *d, const void *q, const void *k_cache,
+                         const void *v_cache, const void *meta, const int32_t *page_table,
+                         const int32_t *seq_lens, int prefix, int window, int budget_tokens,
+                         float scale, int32_t *sel_pages, int32_t *n_sel, void *out,
+                         float *lse, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * csa_decode for callers that cannot allocate device memory.  The paper has
  * no counterpart to this entry point; it exists for deployment: a plugin
  * hosted inside another runtime that owns every device buffer, or a server
@@ -206,12 +223,12 @@ int csa_decode_full(const csa_dims *d, const void *q, const void *k_cache,
  * has no way to provide the workspace csa_decode needs.
  *
  * Same arguments, results and conventions as csa_decode, minus the
- * workspace.  The split-K scratch lives in a 4 MiB __device__ array inside
+ * workspace.  The split-K scratch lives in an 8 MiB __device__ array inside
  * the library (held on every GPU that loads it until the process exits).
  * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
- * routine).  A shape whose scratch would exceed 4 MiB is rejected with
+ * routine).  A shape whose scratch would exceed 8 MiB is rejected with
  * CSA_ERR_WORKSPACE; at D = 128, G = 8 on a 148-SM B200 that is about
- * 700 (sequence, kv-head) units.  The first call on a device looks up the
+ * 560 (sequence, kv-head) units while the decode grid stays at 444 CTAs.  The first call on a device looks up the
  * array's device address (make it before any stream capture).  The call
  * clears the array's flag word on `stream` before the kernels;
  * every call shares the array, so calls that overlap on the GPU race: keep

@@ -26,7 +26,7 @@ DEVFLAG_TIMEOUT = 8
 
 EXPORTS = ("csa_version", "csa_status_string", "csa_workspace_size", "csa_workspace_init",
            "csa_meta_update", "csa_score_select", "csa_decode", "csa_decode_full",
-           "csa_get_device_status", "csa_decode_noalloc")
+           "csa_get_device_status", "csa_decode_noalloc", "csa_sparse_attention")
 
 
 class CsaError(RuntimeError):
@@ -75,8 +75,10 @@ def lib() -> ctypes.CDLL:
         L.csa_decode.argtypes = [D, P, P, P, P, P, P, P, I, I, ctypes.c_float, P, P, P, Z, P]
         L.csa_decode_full.argtypes = [D, P, P, P, P, P, ctypes.c_float, P, P, P, Z, P]
         L.csa_get_device_status.argtypes = [P, P, ctypes.POINTER(I)]
+        L.csa_sparse_attention.argtypes = [D, P, P, P, P, P, P, I, I, I, ctypes.c_float, P, P, P,
+                                           P, P, Z, P]
         for f in ("csa_workspace_init", "csa_meta_update", "csa_score_select", "csa_decode",
-                  "csa_decode_full", "csa_get_device_status"):
+                  "csa_decode_full", "csa_get_device_status", "csa_sparse_attention"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -159,6 +161,22 @@ def decode(d: Dims, q, k_cache, v_cache, page_table, seq_lens, sel, n_sel, prefi
         _stream(stream)))
 
 
+def sparse_attention(d: Dims, q, k_cache, v_cache, meta, page_table, seq_lens, prefix: int,
+                     window: int, budget: int, sel, n_sel, out, ws, lse=None, scale: float = 0.0,
+                     stream=None):
+    """Scoring, top-k selection and the sparse decode in one call (the
+    selection and the decode of the selected pages share a launch when the
+    shape allows)."""
+    bf = torch.bfloat16
+    _check("csa_sparse_attention", lib().csa_sparse_attention(
+        ctypes.byref(d), _ptr(q, bf, "q"), _ptr(k_cache, bf, "k_cache"),
+        _ptr(v_cache, bf, "v_cache"), _ptr(meta, bf, "meta"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        int(prefix), int(window), int(budget), float(scale), _ptr(sel, torch.int32, "sel"),
+        _ptr(n_sel, torch.int32, "n_sel"), _ptr(out, bf, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
 def decode_full(d: Dims, q, k_cache, v_cache, page_table, seq_lens, out, ws, lse=None,
                 scale: float = 0.0, stream=None):
     """Dense decode over every valid token (the unmodified layer)."""
@@ -174,7 +192,7 @@ def decode_noalloc(d: Dims, q, k_cache, v_cache, page_table, seq_lens, sel, n_se
                    window: int, out, lse=None, scale: float = 0.0, stream=None):
     """csa_decode without a workspace, for callers that cannot allocate device
     memory (a plugin inside a runtime that owns all device buffers, a server
-    that reserves the GPU at start-up): the scratch is a fixed 4 MiB array
+    that reserves the GPU at start-up): the scratch is a fixed 8 MiB array
     inside the library, shared by every call on the device, so calls must
     not overlap on the GPU.  Device-side flags of this call are not
     reported."""
@@ -227,12 +245,18 @@ class Layer:
         meta_update(self.d, self.k_cache, self.v_cache, self.meta, self.page_table, self.seq_lens,
                     None, None, n, self.ws, stream)
 
-    def step(self, q, new_k=None, new_v=None, stream=None):
+    def step(self, q, new_k=None, new_v=None, stream=None, fused=False):
         """One decode step.  With new_k/new_v ([B][1][Hkv][D]) the token is
-        appended first; seq_lens must already count it."""
+        appended first; seq_lens must already count it.  fused=True runs
+        scoring, selection and decode as one csa_sparse_attention call."""
         if new_k is not None:
             meta_update(self.d, self.k_cache, self.v_cache, self.meta, self.page_table,
                         self.seq_lens, new_k, new_v, new_k.shape[1], self.ws, stream)
+        if fused:
+            sparse_attention(self.d, q, self.k_cache, self.v_cache, self.meta, self.page_table,
+                             self.seq_lens, self.prefix, self.window, self.budget, self.sel,
+                             self.n_sel, self.out, self.ws, self.lse, stream=stream)
+            return self.out
         score_select(self.d, q, self.meta, self.page_table, self.seq_lens, self.prefix,
                      self.window, self.budget, self.sel, self.n_sel, self.ws, stream=stream)
         decode(self.d, q, self.k_cache, self.v_cache, self.page_table, self.seq_lens, self.sel,

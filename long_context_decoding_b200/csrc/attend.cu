@@ -1,0 +1,256 @@
+// attend.cu -- the top-k selection and the sparse decode in one launch
+// (csa_sparse_attention), after the scoring kernel.
+//
+// Combined sparse attention ("Accelerating Long-Context Decoding in
+// Large-Scale Hybrid LLMs Without Retraining", abstract; "Methodology": the
+// Quest-style top-k pages) attends, per (sequence, kv-head) unit, to the
+// prefix and window tokens and to the tokens of the k best-scoring candidate
+// pages.  Split into separate launches, the part after the selection is a
+// chain of dependent round trips (counts, page lists, page table, K/V) plus a
+// launch; here it shrinks to the page table and the K/V loads.
+//
+// The grid holds two roles, both in clusters of 8 CTAs of 8 warps:
+//   - selection clusters, one per unit (the first 8 * units CTAs): after the
+//     dependency wait (the scores) the cluster selects the unit's top-k pages
+//     (the cluster radix select of select_core.cuh), each CTA receives an
+//     even share of the selected pages, in ascending order, through
+//     distributed shared memory, and its 8 warps attend over that share: the
+//     pages' tokens outside prefix and window (a selected boundary page keeps
+//     its prefix/window tokens in the other role).  Every CTA writes one
+//     partial record of its unit (slot 8u + rank of the second record region).
+//   - prefix/window CTAs (the rest): they attend over every unit's fixed
+//     list (the pages holding prefix or window tokens, masked to those
+//     tokens), flattened and split evenly, and never wait: nothing they read
+//     is written by the scoring kernel, and by the time this grid starts the
+//     kernels before the scoring kernel (the token append among them) have
+//     finished.  They run while the scoring kernel ends and while the
+//     clusters select, when DRAM would otherwise idle.
+// The combine kernel then merges each unit's records of both roles.
+#include "attend_core.cuh"
+#include "common.cuh"
+#include "internal.h"
+#include "select_core.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kFusedUnits = 32;            // units the fused path serves
+constexpr int kFusedItems = kClCap / kCl;  // pages of one CTA's share (2048)
+constexpr int kFusedMinItems = 4 * 8;      // prefix/window pages per CTA, at least
+
+template <int D, int NB>
+struct FusedCfg {
+    static constexpr int kWarps = 8;                    // == kClThreads / 32
+    static constexpr int kBufs = 1;
+    using Tile = TileCfg<D, NB, kWarps, kBufs>;
+    static constexpr size_t kItems = (size_t)kFusedItems * 8;
+    static constexpr size_t kUnits = (size_t)(kFusedUnits + 1) * 4 + (size_t)kFusedUnits * 4;
+    static constexpr size_t kSmem = 1024 /* alignment slack */ + Tile::kStageArea + Tile::kMl +
+                                    kItems + kFusedItems * 4 /* share */ + kUnits;
+};
+static_assert(kClThreads == 256, "the fused kernel runs 8 warps per CTA");
+
+template <int D, int NB>
+__global__ void __cluster_dims__(kCl, 1, 1)
+    __launch_bounds__(kClThreads, (D <= 128 && NB == 1) ? 2 : 1) fused_kernel(FusedParams P) {
+    using C = FusedCfg<D, NB>;
+    using T = typename C::Tile;
+    __shared__ ClShared sh;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // swizzled page buffers need 1024-byte alignment in the shared window
+    uint8_t* stages = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    float* ms = reinterpret_cast<float*>(stages + T::kStageArea);
+    float* ls = ms + C::kWarps * T::kHeads;
+    int2* items = reinterpret_cast<int2*>(ls + C::kWarps * T::kHeads);
+    int* share = reinterpret_cast<int*>(items + kFusedItems);
+    int* uoff = share + kFusedItems;
+    int* ulen = uoff + kFusedUnits + 1;
+
+    const DecodeParams& p = P.d;
+    const int units = p.s.B * p.s.Hkv;
+    const int Hkv = p.s.Hkv, MP = p.s.MP, G = p.s.G;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    AttendArgs A;
+    A.q = p.q;
+    A.k_cache = p.k_cache;
+    A.v_cache = p.v_cache;
+    A.Hq = p.s.Hq;
+    A.Hkv = Hkv;
+    A.G = G;
+    A.prefix = p.prefix;
+    A.window = p.window;
+    A.scale_log2 = p.scale_log2;
+    const size_t rs = record_stride(G, D);
+    int2* rr2 = reinterpret_cast<int2*>(p.rec_range);   // [unit][role]: first, last slot
+    const int n_sel_ctas = kCl * units;
+
+    if ((int)blockIdx.x >= n_sel_ctas) {
+        // ------------------------------------------- prefix/window role
+        const int c0 = (int)blockIdx.x - n_sel_ctas, n0 = (int)gridDim.x - n_sel_ctas;
+        for (int u = tid; u < units; u += kClThreads) {
+            int L = p.seq_lens[u / Hkv];
+            if (L < 0 || L > MP * kPage) L = 0;          // flagged by the scoring kernel
+            ulen[u] = L;
+            uoff[u] = fixed_list(seq_geom(L, p.prefix, p.window), false).total();
+        }
+        __syncthreads();
+        if (warp == 0) {   // exclusive scan (units <= 32: one warp step)
+            const int v = lane < units ? uoff[lane] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (lane < units) uoff[lane] = incl - v;
+            if (lane == 31) uoff[units] = incl;
+        }
+        __syncthreads();
+        const long long T0 = uoff[units];
+        long long want = (T0 + kFusedMinItems - 1) / kFusedMinItems;
+        if (want < 1) want = 1;
+        const int n_cta = (int)(want < (long long)n0 ? want : n0);
+        const long long s = c0 < n_cta ? T0 * c0 / n_cta : T0;
+        const long long e = c0 < n_cta ? T0 * (c0 + 1) / n_cta : T0;
+        if (c0 == 0) {   // units without prefix/window pages: no records
+            for (int u = tid; u < units; u += kClThreads)
+                if (uoff[u + 1] == uoff[u]) rr2[2 * u] = make_int2(0, -1);
+        }
+        if (s >= e) return;
+        for (long long x = s + tid; x < e; x += kClThreads) {
+            const int u = find_unit(uoff, units, x);
+            const SeqGeom sg = seq_geom(ulen[u], p.prefix, p.window);
+            int page = 0, mask = kMaskAll;
+            fixed_item(sg, fixed_list(sg, false), (int)(x - uoff[u]), page, mask);
+            int phys = p.page_table[(size_t)(u / Hkv) * MP + page];
+            if (phys < 0 || phys >= p.s.NPG) {
+                latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
+                phys = -1;
+            }
+            items[x - s] = make_int2(phys, page * 4 + mask);
+        }
+        __syncthreads();
+        const int u_first = find_unit(uoff, units, s);
+        const int u_last = find_unit(uoff, units, e - 1);
+        for (int u = u_first; u <= u_last; ++u) {
+            const long long a = s > uoff[u] ? s : uoff[u];
+            const long long bnd = e < uoff[u + 1] ? e : uoff[u + 1];
+            if (a >= bnd) continue;
+            attend_unit<D, NB, C::kWarps, C::kBufs>(A, u, ulen[u], items, s, a, bnd, stages, ms,
+                                                     ls, p.partials + ((size_t)c0 + u) * rs);
+            const int first = cta_of(uoff[u], T0, n_cta);
+            if (c0 == first && tid == 0)
+                rr2[2 * u] = make_int2(first, cta_of(uoff[u + 1] - 1, T0, n_cta));
+        }
+        return;
+    }
+
+    // ----------------------------------------------- selection role
+    cg::cluster_group cl = cg::this_cluster();
+    const int rank = (int)cl.block_rank();
+    const int u = (int)blockIdx.x / kCl;
+    const int b = u / Hkv;
+    int L = p.seq_lens[b];
+    if (L < 0 || L > MP * kPage) L = 0;                  // flagged by the scoring kernel
+    const SeqGeom sg = seq_geom(L, p.prefix, p.window);
+    const int n = sg.c_hi - sg.c_lo;
+    const int kk = P.k_pages < n ? P.k_pages : n;
+    const int c_lo = sg.c_lo;
+    const int lo = kk * rank / kCl, hi = kk * (rank + 1) / kCl;   // this CTA's share
+    int32_t* out = P.sel + (size_t)u * p.s.max_sel;
+    cluster_select_init(sh);
+    pdl_wait();                 // the scores, and the previous readers of sel
+    pdl_launch_dependents();
+
+    if (kk == n) {              // every candidate fits the budget
+        for (int j = lo + tid; j < hi; j += kClThreads) {
+            share[j - lo] = c_lo + j;
+            out[j] = c_lo + j;
+        }
+    } else if (kk > 0) {
+        cluster_select(cl, sh, P.scores_ws + (size_t)u * MP + c_lo, n, kk, [&](int pos, int i) {
+            out[pos] = c_lo + i;
+            const int dst = cta_of(pos, kk, kCl);
+            int* d = cl.map_shared_rank(share, dst);
+            d[pos - kk * dst / kCl] = c_lo + i;
+        });
+        cl.sync();              // every share is complete
+    }
+    if (rank == 0 && tid == 0) {
+        P.n_sel[u] = kk;
+        rr2[2 * u + 1] = make_int2((kCl - 1) * u, (kCl - 1) * u + kCl - 1);   // slots 8u + r
+    }
+    __syncthreads();
+    const int cnt = hi - lo;
+    for (int j = tid; j < cnt; j += kClThreads) {
+        const int page = share[j];
+        int phys = p.page_table[(size_t)b * MP + page];
+        if (phys < 0 || phys >= p.s.NPG) {
+            latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
+            phys = -1;
+        }
+        items[j] = make_int2(phys, page * 4 + kMaskRest);
+    }
+    __syncthreads();
+    attend_unit<D, NB, C::kWarps, C::kBufs>(A, u, L, items, 0, 0, cnt, stages, ms, ls,
+                                             p.partials + p.phase_floats +
+                                                 ((size_t)kCl * u + rank) * rs);
+}
+
+template <int D, int NB>
+cudaError_t launch_fused_t(const FusedParams& p, cudaStream_t st) {
+    using C = FusedCfg<D, NB>;
+    auto kern = fused_kernel<D, NB>;
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)C::kSmem);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = 1;
+    }
+    const int units = p.d.s.B * p.d.s.Hkv;
+    const int grid = kCl * units + p.n0;
+    cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kClThreads), C::kSmem, st, p);
+    if (e != cudaSuccess) return e;
+    return launch_combine(p.d, st);
+}
+
+}  // namespace
+
+// The fused path serves up to 32 units, with at most kClCap candidates per
+// unit (the cluster select's capacity) and at least one page to select.
+bool fused_eligible(const Shape& s, int prefix, int window, int k_pages) {
+    const long long n_max = (long long)s.MP - prefix / kPage - window / kPage;
+    return k_pages > 0 && (long long)s.B * s.Hkv <= kFusedUnits && n_max <= kClCap;
+}
+
+// CTAs of the prefix/window role: what stays of the resident capacity beside
+// the selection clusters, at least enough that no slice exceeds the item
+// capacity, and a whole number of clusters.
+int fused_phase0_ctas(const Shape& s) {
+    const long long units = (long long)s.B * s.Hkv;
+    const int per_sm = (s.D <= 128 && s.G <= 8) ? 2 : 1;
+    long long n0 = (long long)per_sm * device_sm_count() - kCl * units;
+    const long long cap = (units * (s.MP + 2) + kFusedItems - 1) / kFusedItems;
+    if (n0 < cap) n0 = cap;
+    if (n0 < kCl) n0 = kCl;
+    n0 = (n0 + kCl - 1) / kCl * kCl;
+    return (int)(n0 < (1ll << 30) ? n0 : (1ll << 30));
+}
+
+cudaError_t launch_fused(const FusedParams& p, cudaStream_t st) {
+    const int nb = p.d.s.G > 8 ? 2 : 1;
+    switch (p.d.s.D * 10 + nb) {
+        case 641: return launch_fused_t<64, 1>(p, st);
+        case 642: return launch_fused_t<64, 2>(p, st);
+        case 1281: return launch_fused_t<128, 1>(p, st);
+        case 1282: return launch_fused_t<128, 2>(p, st);
+        case 2561: return launch_fused_t<256, 1>(p, st);
+        case 2562: return launch_fused_t<256, 2>(p, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace csa

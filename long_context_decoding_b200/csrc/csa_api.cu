@@ -63,7 +63,13 @@ WsLayout workspace_layout(const Shape& s) {
     w.scores = off;
     off = align_up(off + 4 * units * (size_t)s.MP, 256);
     w.partials = off;
-    w.dec_slots = (size_t)decode_grid(s) + units;
+    // record slots per phase: a decode CTA or a prefix/window CTA of the fused
+    // kernel per slot plus one per unit, or the 8 CTAs of each unit's cluster
+    size_t slots = (size_t)decode_grid(s) + units;
+    const size_t fused = (size_t)fused_phase0_ctas(s) + units;
+    if (fused > slots) slots = fused;
+    if (8 * units > slots) slots = 8 * units;
+    w.dec_slots = slots;
     off = align_up(off + 2 * 4 * w.dec_slots * decode_record_floats(s), 256);
     w.total = off;
     return w;
@@ -310,6 +316,99 @@ int csa_decode_full(const csa_dims* d, const void* q, const void* k_cache, const
                     float* lse, void* workspace, size_t workspace_bytes, void* stream) {
     return decode_common(d, q, k_cache, v_cache, page_table, seq_lens, nullptr, nullptr, 0, 0, 1,
                          scale, out, lse, workspace, workspace_bytes, stream);
+}
+
+int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
+                         const void* v_cache, const void* meta, const int32_t* page_table,
+                         const int32_t* seq_lens, int prefix, int window, int budget_tokens,
+                         float scale, int32_t* sel_pages, int32_t* n_sel, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    Shape s;
+    int rc = check_dims(d, &s);
+    if (rc != CSA_OK) return rc;
+    CSA_REQUIRE(q);
+    CSA_REQUIRE(k_cache);
+    CSA_REQUIRE(v_cache);
+    CSA_REQUIRE(meta);
+    CSA_REQUIRE(page_table);
+    CSA_REQUIRE(seq_lens);
+    CSA_REQUIRE(sel_pages);
+    CSA_REQUIRE(n_sel);
+    CSA_REQUIRE(out);
+    CSA_OPTIONAL(lse);
+    if (prefix < 0 || window < 0 || budget_tokens < 0) return CSA_ERR_INVALID_ARG;
+    const int k_pages = budget_tokens / kPage;
+    if (k_pages > s.max_sel) return CSA_ERR_INVALID_ARG;
+    if (!(scale == scale) || isinf(scale)) return CSA_ERR_INVALID_ARG;
+    WsLayout w;
+    rc = check_ws(s, workspace, workspace_bytes, &w);
+    if (rc != CSA_OK) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    note_stream_call(stream, kCallOther);
+
+    ScoreParams sp;
+    sp.q = static_cast<const uint16_t*>(q);
+    sp.meta = static_cast<const uint16_t*>(meta);
+    sp.page_table = page_table;
+    sp.seq_lens = seq_lens;
+    sp.prefix = prefix;
+    sp.window = window;
+    sp.scores_ws = at<float>(workspace, w.scores);
+    sp.scores_out = nullptr;
+    sp.flags = at<uint32_t>(workspace, w.flags);
+    sp.s = s;
+    if (k_pages > 0) {
+        rc = launch_status(launch_score(sp, st));
+        if (rc != CSA_OK) return rc;
+    }
+
+    DecodeParams dp;
+    dp.q = sp.q;
+    dp.k_cache = static_cast<const uint16_t*>(k_cache);
+    dp.v_cache = static_cast<const uint16_t*>(v_cache);
+    dp.page_table = page_table;
+    dp.seq_lens = seq_lens;
+    dp.sel = sel_pages;
+    dp.n_sel = n_sel;
+    dp.prefix = prefix;
+    dp.window = window;
+    dp.dense = 0;
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)s.D);
+    dp.scale_log2 = sc * 1.4426950408889634f;
+    dp.out = static_cast<uint16_t*>(out);
+    dp.lse = lse;
+    dp.flags = sp.flags;
+    dp.rec_range = at<int4>(workspace, w.rec_range);
+    dp.partials = at<float>(workspace, w.partials);
+    dp.phase_floats = w.dec_slots * decode_record_floats(s);
+    dp.s = s;
+
+    if (fused_eligible(s, prefix, window, k_pages)) {
+        FusedParams fp;
+        fp.d = dp;
+        fp.d.early = 1;
+        fp.scores_ws = sp.scores_ws;
+        fp.k_pages = k_pages;
+        fp.sel = sel_pages;
+        fp.n_sel = n_sel;
+        fp.n0 = fused_phase0_ctas(s);
+        return launch_status(launch_fused(fp, st));
+    }
+    SelectParams lp;
+    lp.scores_ws = sp.scores_ws;
+    lp.seq_lens = seq_lens;
+    lp.prefix = prefix;
+    lp.window = window;
+    lp.k_pages = k_pages;
+    lp.sel = sel_pages;
+    lp.n_sel = n_sel;
+    lp.flags = sp.flags;
+    lp.smem_keys = 0;
+    lp.s = s;
+    rc = launch_status(launch_select(lp, st));
+    if (rc != CSA_OK) return rc;
+    dp.early = 1;   // our own scoring and selection kernels are the ones ahead
+    return launch_status(launch_decode(dp, st));
 }
 
 int csa_get_device_status(void* workspace, void* stream, int* flags_out) {

@@ -86,6 +86,23 @@ struct DecodeParams {
     Shape s;
 };
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st);
+
+// ---------------------------------------------------------------- fused
+// Selection + decode in one launch (csa_sparse_attention): clusters of 8
+// CTAs select the top-k pages of one unit each and attend over them; more
+// CTAs of the same grid attend over the prefix and window pages meanwhile.
+struct FusedParams {
+    DecodeParams d;          // q, caches, geometry, outputs, workspace records
+    const float* scores_ws;  // [units][MP] Quest scores of the candidates
+    int k_pages;
+    int32_t* sel;            // [units][max_sel] selected pages (output)
+    int32_t* n_sel;          // [units] (output)
+    int n0;                  // CTAs of the prefix/window role (a multiple of 8)
+};
+bool fused_eligible(const Shape& s, int prefix, int window, int k_pages);
+int fused_phase0_ctas(const Shape& s);
+cudaError_t launch_fused(const FusedParams& p, cudaStream_t st);
 
 // Kind of the last kernel-launching call issued on a stream (host side).
 // csa_decode streams the prefix/window pages before the dependency wait only

@@ -32,7 +32,7 @@
 namespace csa {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;   // 4 MiB per GPU
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;   // 8 MiB per GPU
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;

@@ -2,6 +2,7 @@
 same seeded inputs (metadata bit-exact, scores to fp32 accuracy, selection by
 the band rule, attention within max-abs 2e-2 / mean-abs 2e-3 of fp32)."""
 import math
+from dataclasses import replace
 
 import numpy as np
 import pytest
@@ -229,3 +230,127 @@ def test_fixed_pages_streamed_before_the_selection_ends(cuda):
         assert torch.equal(out_e, out_w)
         assert torch.equal(lse_e, lse_w)
     assert csa.device_status(run.ws) == 0
+
+
+# ---------------------------------------------------------------- one-call path
+def sparse_call(run: Run):
+    """csa_sparse_attention on the run's layer: (sel, n_sel, out, lse)."""
+    d, c = run.d, run.c
+    sel = torch.full((d.B, d.Hkv, d.max_sel), -7, dtype=torch.int32, device=c.q.device)
+    nsel = torch.full((d.B, d.Hkv), -7, dtype=torch.int32, device=c.q.device)
+    out = torch.full((d.B, d.Hq, d.D), float("nan"), dtype=torch.bfloat16, device=c.q.device)
+    lse = torch.full((d.B, d.Hq), float("nan"), dtype=torch.float32, device=c.q.device)
+    csa.sparse_attention(d, c.q, c.k_cache, c.v_cache, run.layer.meta, c.page_table, c.seq_lens,
+                         run.prefix, run.window, run.budget, sel, nsel, out, run.ws, lse)
+    return sel, nsel, out, lse
+
+
+def check_one_call(run: Run, oracle_too=True):
+    """The one-call path selects exactly what csa_score_select selects, attends
+    like csa_decode on that selection, and, where the oracle's selection is
+    unambiguous for every unit, matches the oracle."""
+    run.gpu_meta()
+    sel_f, nsel_f, out_f, lse_f = sparse_call(run)
+    run.gpu_select(scores=False)
+    out_s, lse_s = run.gpu_decode(run.layer.sel, run.layer.n_sel)
+    torch.cuda.synchronize()
+    assert csa.device_status(run.ws) == 0
+    assert torch.equal(nsel_f, run.layer.n_sel)
+    for b in range(run.d.B):
+        for g in range(run.d.Hkv):
+            k = int(nsel_f[b, g])
+            assert torch.equal(sel_f[b, g, :k], run.layer.sel[b, g, :k]), f"unit ({b},{g})"
+    # the same attention, split differently: bf16 output rounding apart
+    err = (out_f.float() - out_s.float()).abs()
+    assert torch.isfinite(out_f.float()).all()
+    assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3
+    fin = torch.isfinite(lse_s)
+    assert torch.equal(torch.isfinite(lse_f), fin)
+    torch.testing.assert_close(lse_f[fin], lse_s[fin], rtol=1e-4, atol=1e-3)
+    if oracle_too:
+        # selection by the band rule; then, in every unit whose selection is
+        # the oracle's own, the attention output of its heads against the oracle
+        ref = run.oracle_step()
+        check_selection(sel_f, nsel_f, ref["scores"], ref["sel"], ref["nsel"])
+        gs, gn = sel_f.cpu().numpy(), nsel_f.cpu().numpy()
+        G = run.d.Hq // run.d.Hkv
+        same = 0
+        for b in range(run.d.B):
+            for g in range(run.d.Hkv):
+                k = int(gn[b, g])
+                if not np.array_equal(gs[b, g, :k], ref["sel"][b, g, :k]):
+                    continue
+                same += 1
+                h = slice(g * G, (g + 1) * G)
+                assert_out_close(out_f[b, h], lse_f[b, h], ref["out"][b, h], ref["lse"][b, h],
+                                 f"one-call decode, unit ({b},{g})")
+        return same
+    return None
+
+
+@pytest.mark.parametrize("w", [wl.TINY, wl.CTX32K, wl.CTX64K], ids=lambda w: w.name)
+def test_one_call_parity(w, cuda):
+    same = check_one_call(Run(wl.make_case(w, cuda)))
+    if w is wl.CTX32K:
+        assert same >= 1
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_one_call_output_against_oracle(D, cuda):
+    """k equal to the number of q-aligned planted pages, one query head per
+    kv-head (the plant then stands about 5 sigma above the random pages'
+    bounds): the oracle's top-k is unambiguous in most units, and in each of
+    them the one-call output is compared with the oracle's attention.  (With 8
+    heads per group a plant along the group's summed query stands out much
+    less.)"""
+    G = 1
+    w = wl.Workload("planted_exact", B=3, Hq=2 * G, Hkv=2, D=D, seq_lens=(20000, 13001, 7777),
+                    prefix=64, window=512, budget=16 * 12, planted=12, seed=11)
+    same = check_one_call(Run(wl.make_case(w, cuda)))
+    assert same >= 4
+
+
+@pytest.mark.parametrize("G", [1, 8, 16])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_one_call_group_sizes_and_head_dims(G, D, cuda):
+    w = small(B=2, Hq=2 * G, Hkv=2, D=D, lens=(3000, 2049), prefix=40, window=100, budget=480)
+    check_one_call(Run(wl.make_case(w, cuda)))
+
+
+@pytest.mark.parametrize("lens,P,W,budget", [
+    ((1000, 777), 20, 50, 160),        # ragged, partial boundary pages
+    ((4096, 16), 0, 0, 256),           # no prefix or window; a one-page sequence
+    ((700, 699), 8, 8, 16 * 44),       # budget covers every candidate
+    ((513, 2000), 512, 1, 32),         # prefix covers the first sequence
+    ((0, 300), 16, 16, 64),            # an empty sequence
+    ((333, 4000), 17, 33, 0),          # budget 0: separate kernels
+])
+def test_one_call_edge_geometry(lens, P, W, budget, cuda):
+    w = small(lens=lens, prefix=P, window=W, budget=budget)
+    check_one_call(Run(wl.make_case(w, cuda)))
+
+
+def test_one_call_many_units_uses_separate_kernels(cuda):
+    """More than 32 (sequence, kv-head) units: the separate-kernel path."""
+    w = small(B=20, Hq=16, Hkv=2, lens=tuple(900 + 37 * i for i in range(20)), prefix=16,
+              window=64, budget=256)
+    check_one_call(Run(wl.make_case(w, cuda)), oracle_too=False)
+
+
+def test_one_call_repeated_and_after_appends(cuda):
+    """Back-to-back one-call steps with appends in between, no host syncs."""
+    w = replace(wl.CTX32K, steps=4)
+    case = wl.make_case(w, cuda)
+    run = Run(case)
+    run.gpu_meta()
+    outs = []
+    for s in range(4):
+        nk, nv = wl.step_tokens(case, s)[1:]
+        case.seq_lens += 1
+        csa.meta_update(run.d, case.k_cache, case.v_cache, run.layer.meta, case.page_table,
+                        case.seq_lens, nk, nv, 1, run.ws)
+        outs.append(sparse_call(run))
+    torch.cuda.synchronize()
+    assert csa.device_status(run.ws) == 0
+    run.refresh_host()
+    check_one_call(run, oracle_too=False)
