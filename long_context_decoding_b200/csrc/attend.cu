@@ -36,7 +36,7 @@ namespace {
 
 constexpr int kFusedUnits = 32;            // units the fused path serves
 constexpr int kFusedItems = kClCap / kCl;  // pages of one CTA's share (2048)
-constexpr int kFusedMinItems = 4 * 8;      // prefix/window pages per CTA, at least
+constexpr int kFusedMinItems = 4 * 8;      // prefix/window pages per CTA, at least (16 measured slower)
 
 template <int D, int NB>
 struct FusedCfg {
@@ -158,7 +158,11 @@ __global__ void __cluster_dims__(kCl, 1, 1)
     const int c_lo = sg.c_lo;
     const int lo = kk * rank / kCl, hi = kk * (rank + 1) / kCl;   // this CTA's share
     int32_t* out = P.sel + (size_t)u * p.s.max_sel;
-    cluster_select_init(sh);
+    cluster_select_begin(sh);
+    if (tid < G * D / 64) {     // this unit's queries (a caller input) into L1
+        const uint16_t* qrow = p.q + ((size_t)b * p.s.Hq + (size_t)(u % Hkv) * G) * D + tid * 64;
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(qrow));
+    }
     pdl_wait();                 // the scores, and the previous readers of sel
     pdl_launch_dependents();
 
@@ -168,16 +172,20 @@ __global__ void __cluster_dims__(kCl, 1, 1)
             out[j] = c_lo + j;
         }
     } else if (kk > 0) {
-        cluster_select(cl, sh, P.scores_ws + (size_t)u * MP + c_lo, n, kk, [&](int pos, int i) {
-            out[pos] = c_lo + i;
-            const int dst = cta_of(pos, kk, kCl);
-            int* d = cl.map_shared_rank(share, dst);
-            d[pos - kk * dst / kCl] = c_lo + i;
-        });
+        uint32_t kmin, kmax;
+        key_range(P.keyrange[u], kmin, kmax);
+        cluster_select(cl, sh, P.scores_ws + (size_t)u * MP + c_lo, n, kk, kmin, kmax,
+                       [&](int pos, int i) {
+                           out[pos] = c_lo + i;
+                           const int dst = cta_of(pos, kk, kCl);
+                           int* d = cl.map_shared_rank(share, dst);
+                           d[pos - kk * dst / kCl] = c_lo + i;
+                       });
         cl.sync();              // every share is complete
     }
-    if (rank == 0 && tid == 0) {
+    if (rank == 0 && tid == 0) {   // every CTA read the key range before the last barrier
         P.n_sel[u] = kk;
+        P.keyrange[u] = make_uint2(0u, 0u);
         rr2[2 * u + 1] = make_int2((kCl - 1) * u, (kCl - 1) * u + kCl - 1);   // slots 8u + r
     }
     __syncthreads();

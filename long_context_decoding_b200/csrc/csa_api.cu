@@ -60,6 +60,8 @@ WsLayout workspace_layout(const Shape& s) {
     off = align_up(off + 4, 256);
     w.rec_range = off;
     off = align_up(off + 16 * units, 256);
+    w.keyrange = off;
+    off = align_up(off + 8 * units, 256);
     w.scores = off;
     off = align_up(off + 4 * units * (size_t)s.MP, 256);
     w.partials = off;
@@ -229,6 +231,7 @@ int csa_score_select(const csa_dims* d, const void* q, const void* meta,
     sp.window = window;
     sp.scores_ws = at<float>(workspace, w.scores);
     sp.scores_out = scores_out;
+    sp.keyrange = at<uint2>(workspace, w.keyrange);
     sp.flags = at<uint32_t>(workspace, w.flags);
     sp.s = s;
     if (k_pages > 0 || scores_out) {
@@ -246,6 +249,7 @@ int csa_score_select(const csa_dims* d, const void* q, const void* meta,
     lp.k_pages = k_pages;
     lp.sel = sel_pages;
     lp.n_sel = n_sel;
+    lp.keyrange = sp.keyrange;
     lp.flags = sp.flags;
     lp.smem_keys = 0;
     lp.s = s;
@@ -355,6 +359,7 @@ int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
     sp.window = window;
     sp.scores_ws = at<float>(workspace, w.scores);
     sp.scores_out = nullptr;
+    sp.keyrange = at<uint2>(workspace, w.keyrange);
     sp.flags = at<uint32_t>(workspace, w.flags);
     sp.s = s;
     if (k_pages > 0) {
@@ -391,6 +396,7 @@ int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
         fp.k_pages = k_pages;
         fp.sel = sel_pages;
         fp.n_sel = n_sel;
+        fp.keyrange = sp.keyrange;
         fp.n0 = fused_phase0_ctas(s);
         return launch_status(launch_fused(fp, st));
     }
@@ -402,6 +408,7 @@ int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
     lp.k_pages = k_pages;
     lp.sel = sel_pages;
     lp.n_sel = n_sel;
+    lp.keyrange = sp.keyrange;
     lp.flags = sp.flags;
     lp.smem_keys = 0;
     lp.s = s;

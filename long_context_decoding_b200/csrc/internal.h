@@ -12,6 +12,7 @@ namespace csa {
 struct WsLayout {
     size_t flags;          // uint32 device flag word
     size_t rec_range;      // int4 [units]
+    size_t keyrange;       // uint2 [units]: ~min and max order key of the scores
     size_t scores;         // fp32 [B][Hkv][max_pages]
     size_t partials;       // fp32 [2][dec_slots][decode_record_floats]
     size_t dec_slots;      // partial records available per decode phase
@@ -46,6 +47,7 @@ struct ScoreParams {
     int prefix, window;
     float* scores_ws;       // [B][Hkv][MP]
     float* scores_out;      // nullable
+    uint2* keyrange;        // [units] merged with atomicMax: ~min key, max key
     uint32_t* flags;
     Shape s;
 };
@@ -58,6 +60,7 @@ struct SelectParams {
     int prefix, window, k_pages;
     int32_t* sel;
     int32_t* n_sel;
+    uint2* keyrange;        // [units] from the scoring kernel; reset to zero here
     uint32_t* flags;
     int smem_keys;          // keys that fit in the dynamic shared memory (set by the launcher)
     Shape s;
@@ -98,6 +101,7 @@ struct FusedParams {
     int k_pages;
     int32_t* sel;            // [units][max_sel] selected pages (output)
     int32_t* n_sel;          // [units] (output)
+    uint2* keyrange;         // [units] from the scoring kernel; reset to zero here
     int n0;                  // CTAs of the prefix/window role (a multiple of 8)
 };
 bool fused_eligible(const Shape& s, int prefix, int window, int k_pages);

@@ -199,6 +199,8 @@ score_kernel(ScoreParams p) {
     int cur_unit = -1;
     walk.start(s, e);
     TileInfo t;
+    int kr_unit = -1;                        // key range of this warp's current unit
+    uint32_t kr_nmin = 0u, kr_max = 0u;
     for (int j = 0; walk.next(t); ++j) {
         if (j % C::kWarps != warp) continue;
         const int b = t.unit / Hkv, g = t.unit % Hkv;
@@ -271,14 +273,33 @@ score_kernel(ScoreParams p) {
         m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
         m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
         const int row = tq == 0 ? gq : gq + 8;
-        if (tq < 2 && row < t.count) {
-            const bool ok = tq == 0 ? ok0 : ok8;
+        const bool has = tq < 2 && row < t.count;
+        const bool ok = tq == 0 ? ok0 : ok8;
+        const float v = ok ? (tq == 0 ? m0 : m8) : -INFINITY;
+        if (has) {
             if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
-            const float v = ok ? (tq == 0 ? m0 : m8) : -INFINITY;
             const size_t o = (size_t)t.unit * MP + t.first + row;
             p.scores_ws[o] = v;
             if (p.scores_out) p.scores_out[o] = v;
         }
+        // the unit's key range for the selection (min kept as ~key, so that
+        // both ends merge with atomicMax from a zeroed word), published once
+        // per warp and unit: per-tile atomics on one word serialise in L2
+        const uint32_t key = order_key(v);
+        if (t.unit != kr_unit) {
+            if (lane == 0 && kr_unit >= 0) {
+                atomicMax(&p.keyrange[kr_unit].x, kr_nmin);
+                atomicMax(&p.keyrange[kr_unit].y, kr_max);
+            }
+            kr_unit = t.unit;
+            kr_nmin = kr_max = 0u;
+        }
+        kr_nmin = max(kr_nmin, __reduce_max_sync(0xffffffffu, has ? ~key : 0u));
+        kr_max = max(kr_max, __reduce_max_sync(0xffffffffu, has ? key : 0u));
+    }
+    if (lane == 0 && kr_unit >= 0) {
+        atomicMax(&p.keyrange[kr_unit].x, kr_nmin);
+        atomicMax(&p.keyrange[kr_unit].y, kr_max);
     }
 }
 

@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectParams p) 
     // scores (and the previous readers of sel) belong to earlier kernels
     pdl_wait();
     pdl_launch_dependents();
+    if (tid == 0) p.keyrange[u] = make_uint2(0u, 0u);   // left by the scoring kernel, unused
 
     if (kk == n) {                              // every candidate fits the budget
         for (int i = tid; i < n; i += kSelThreads) out[i] = sg.c_lo + i;
@@ -303,24 +304,35 @@ select_cluster_kernel(SelectParams p) {
     const int n = sg.c_hi - sg.c_lo;
     const int kk = p.k_pages < n ? p.k_pages : n;
     int32_t* out = p.sel + (size_t)u * p.s.max_sel;
-    cluster_select_init(sh);
+    cluster_select_begin(sh);
     pdl_wait();                 // scores and the previous readers of sel
     pdl_launch_dependents();
 
     if (kk == n) {              // every candidate fits the budget
         for (int i = rank * kClThreads + tid; i < n; i += kCl * kClThreads) out[i] = sg.c_lo + i;
-        if (rank == 0 && tid == 0) p.n_sel[u] = n;
+        if (rank == 0 && tid == 0) {
+            p.n_sel[u] = n;
+            p.keyrange[u] = make_uint2(0u, 0u);
+        }
         return;
     }
     if (kk == 0 || n > kClCap) {
-        if (rank == 0 && tid == 0) p.n_sel[u] = 0;
-        if (n > kClCap && rank == 0 && tid == 0) latch_flag(p.flags, CSA_DEVFLAG_BAD_SELECTION);
+        if (rank == 0 && tid == 0) {
+            p.n_sel[u] = 0;
+            p.keyrange[u] = make_uint2(0u, 0u);
+            if (n > kClCap) latch_flag(p.flags, CSA_DEVFLAG_BAD_SELECTION);
+        }
         return;
     }
     const int c_lo = sg.c_lo;
-    cluster_select(cl, sh, p.scores_ws + (size_t)u * MP + c_lo, n, kk,
+    uint32_t kmin, kmax;
+    key_range(p.keyrange[u], kmin, kmax);
+    cluster_select(cl, sh, p.scores_ws + (size_t)u * MP + c_lo, n, kk, kmin, kmax,
                    [&](int pos, int i) { out[pos] = c_lo + i; });
-    if (rank == 0 && tid == 0) p.n_sel[u] = kk;
+    if (rank == 0 && tid == 0) {   // every CTA read the range before the last barrier
+        p.n_sel[u] = kk;
+        p.keyrange[u] = make_uint2(0u, 0u);
+    }
 }
 
 }  // namespace

@@ -48,30 +48,52 @@ constexpr int kClPasses = 4;                        // at most four 8-bit digits
 
 struct ClShared {
     uint32_t hist[kClPasses][256];   // rank 0: merged histogram of each pass
-    uint32_t local[256];             // this CTA's histogram / copy of the merged one
-    uint32_t kmin, kmax;             // rank 0: cluster min / max
-    uint32_t cgt[kCl], ceq[kCl];     // rank 0: per-CTA (above, equal) counts
+    uint32_t local[256];             // this CTA's histogram
+    uint32_t cgt[kCl], ceq[kCl];     // every CTA: the (above, equal) counts of each rank
     uint32_t red[kClWarps], wgt[kClWarps], weq[kClWarps];
     uint32_t digit, gt, cnt;
 };
 
-// Rank 0's merge buffers start empty; call before the first cluster barrier
-// (the first barrier of cluster_select publishes them).
-__device__ __forceinline__ void cluster_select_init(ClShared& sh) {
+// Split cluster barrier (arrive now, wait later) with release / acquire
+// semantics on the cluster's shared memory.
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Empties rank 0's merge buffers and arrives at the cluster barrier that
+// publishes them; call before the dependency wait (it touches only this
+// CTA's shared memory).  cluster_select waits on that barrier before its
+// first remote access.
+__device__ __forceinline__ void cluster_select_begin(ClShared& sh) {
     for (int i = threadIdx.x; i < kClPasses * 256; i += kClThreads) (&sh.hist[0][0])[i] = 0;
-    if (threadIdx.x == 0) {
-        sh.kmin = 0xffffffffu;
-        sh.kmax = 0u;
+    __syncthreads();
+    cluster_arrive();
+}
+
+// Key range of a unit as published by the scoring kernel: x = ~min key,
+// y = max key (both merged with atomicMax, so zero means "nothing yet").
+// A range nobody wrote becomes the full key space, which is still exact.
+__device__ __forceinline__ void key_range(uint2 r, uint32_t& kmin, uint32_t& kmax) {
+    kmin = ~r.x;
+    kmax = r.y;
+    if (kmin > kmax) {
+        kmin = 0u;
+        kmax = 0xffffffffu;
     }
 }
 
-// Selects the kk largest of the n scores sc[0, n) (0 < kk < n <= kClCap)
-// with the CTAs of the cluster; calls emit(pos, i) for every selected
-// candidate i in this CTA's share, pos being its rank in ascending index
-// order.  Called by every thread of all kCl CTAs.
+// Selects the kk largest of the n scores sc[0, n) (0 < kk < n <= kClCap),
+// whose order keys all lie in [kmin, kmax], with the CTAs of the cluster;
+// calls emit(pos, i) for every selected candidate i in this CTA's share, pos
+// being its rank in ascending index order.  Called by every thread of all
+// kCl CTAs after cluster_select_begin; ends with a cluster barrier, after
+// which no CTA reads another's shared memory.
 template <typename Emit>
 __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float* sc, int n, int kk,
-                               Emit emit) {
+                               uint32_t kmin, uint32_t kmax, Emit emit) {
     const int rank = (int)cl.block_rank();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     ClShared* sh0 = cl.map_shared_rank(&sh, 0);
@@ -84,39 +106,12 @@ __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float*
     const int wlo = clo + warp * wspan;
     const int whi = wlo + wspan < chi ? wlo + wspan : chi;
     uint32_t kr[kClKeys];
-    float v[kClKeys];
 #pragma unroll
     for (int j = 0; j < kClKeys; ++j) {
         const int i = wlo + 32 * j + lane;
-        v[j] = __ldcg(sc + (i < whi ? i : 0));
+        kr[j] = order_key(__ldcg(sc + (i < whi ? i : 0)));
     }
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-#pragma unroll
-    for (int j = 0; j < kClKeys; ++j) {
-        kr[j] = order_key(v[j]);
-        if (wlo + 32 * j + lane < whi) {
-            kmin = min(kmin, kr[j]);
-            kmax = max(kmax, kr[j]);
-        }
-    }
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    if (lane == 0) {
-        sh.red[warp] = kmin;
-        sh.wgt[warp] = kmax;
-    }
-    cl.sync();                  // rank 0 buffers initialised everywhere; warp results in
-    if (warp == 0) {
-        kmin = __reduce_min_sync(0xffffffffu, lane < kClWarps ? sh.red[lane] : 0xffffffffu);
-        kmax = __reduce_max_sync(0xffffffffu, lane < kClWarps ? sh.wgt[lane] : 0u);
-        if (lane == 0) {
-            atomicMin(&sh0->kmin, kmin);
-            atomicMax(&sh0->kmax, kmax);
-        }
-    }
-    cl.sync();
-    kmin = sh0->kmin;
-    kmax = sh0->kmax;
+    cluster_wait();             // rank 0's buffers are empty everywhere
 
     uint32_t pmask, pval;
     uint32_t remaining = (uint32_t)kk;
@@ -172,7 +167,8 @@ __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float*
     }
     const uint32_t eq_take = take_all ? 0xffffffffu : remaining;
 
-    // compaction: per-warp, per-CTA and per-cluster prefixes of (above, equal)
+    // compaction: per-warp, per-CTA and per-cluster prefixes of (above, equal);
+    // every CTA sends its totals to every CTA, so one barrier suffices
     uint32_t cgt = 0, ceq = 0;
 #pragma unroll
     for (int j = 0; j < kClKeys; ++j) {
@@ -188,18 +184,18 @@ __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float*
     __syncthreads();
     uint32_t gt_base = warp_prefix(sh.wgt, kClWarps);
     uint32_t eq_base = warp_prefix(sh.weq, kClWarps);
-    if (tid == kClThreads - 1) {     // this CTA's totals to rank 0
-        sh0->cgt[rank] = gt_base + cgt;
-        sh0->ceq[rank] = eq_base + ceq;
+    if (tid >= kClThreads - kCl) {   // last warp (its gt_base + cgt is the CTA's total)
+        ClShared* dst = cl.map_shared_rank(&sh, tid - (kClThreads - kCl));
+        dst->cgt[rank] = gt_base + cgt;
+        dst->ceq[rank] = eq_base + ceq;
     }
-    cl.sync();
+    cl.sync();                  // counts everywhere; no remote reads after this
     {
-        const uint32_t x = lane < kCl && lane < rank ? sh0->cgt[lane] : 0u;
-        const uint32_t y = lane < kCl && lane < rank ? sh0->ceq[lane] : 0u;
+        const uint32_t x = lane < kCl && lane < rank ? sh.cgt[lane] : 0u;
+        const uint32_t y = lane < kCl && lane < rank ? sh.ceq[lane] : 0u;
         gt_base += __reduce_add_sync(0xffffffffu, x);
         eq_base += __reduce_add_sync(0xffffffffu, y);
     }
-    cl.sync();                  // rank 0 stays alive until every CTA has read it
     const uint32_t lt_mask = (1u << lane) - 1u;
 #pragma unroll
     for (int j = 0; j < kClKeys; ++j) {
