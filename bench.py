@@ -287,10 +287,16 @@ class Stack:
     def launches_per_step(self) -> int:
         """Kernels of one step: per layer the metadata update, then the scoring
         kernel, the fused selection + decode kernel and the split-K combine
-        (or, with nothing to select, the selection, decode and combine)."""
+        when the one-call path applies (k >= 1, at most 32 units, at most
+        16384 candidates per unit), else scoring (k >= 1), selection, decode
+        and combine."""
+        w = self.w
         n = 0
         for lay in self.layers:
-            n += 1 + 3
+            k = lay.budget // 16
+            n_max = w.max_pages - lay.prefix // 16 - lay.window // 16
+            fused = k > 0 and w.B * w.Hkv <= 32 and n_max <= 16384
+            n += 1 + (3 if fused else (1 if k > 0 else 0) + 3)
         return n
 
     def graph(self, fn):
