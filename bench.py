@@ -65,6 +65,10 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=0,
                     help="use only the first N layers (small cases for ncu captures)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the step: sparse (one call) vs dense decode over uniform "
+                         "lengths 4k..256k and budgets 0/1024/4096/all, with a byte-based "
+                         "cost-model fit; prints one JSON line")
     return ap.parse_args()
 
 
@@ -496,10 +500,11 @@ def e2e(st: Stack, K: int, W: int, dist: Dist):
 
 def secondary_64k(dev, dist: Dist):
     """The 64k single-layer workload: one layer step (one
-    csa_sparse_attention call: score, select, decode; no append) per graph; a 256 MB read between replays flushes L2
-    (the layer itself moves only ~84 MB).  The flush reads rather than
-    writes, so that no dirty L2 lines are written back during the timed
-    replay."""
+    csa_sparse_attention call: score, select, decode; no append) per graph;
+    a 256 MB read before every replay flushes L2 (the layer itself moves only
+    ~84 MB), and batches of replays are timed (graph_time).  The flush reads
+    rather than writes, so that no dirty L2 lines are written back during the
+    timed replay."""
     from long_context_decoding_b200 import csa
     w = wl.CTX64K
     c = wl.make_case(w, dev)
@@ -508,65 +513,142 @@ def secondary_64k(dev, dist: Dist):
                     w.budget)
     lay.rebuild_meta()
     scrub = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MB
-
-    def body():
-        lay.step(c.q, fused=True)
-
-    body()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        with torch.cuda.graph(g, stream=s):
-            body()
-    torch.cuda.current_stream().wait_stream(s)
-    times = []
     sink = torch.zeros((), device=dev)
-    for i in range(30):
+
+    def flush():
         torch.sum(scrub, dim=0, out=sink)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        g.replay()
-        b.record()
-        torch.cuda.synchronize()
-        if i >= 5:
-            times.append(a.elapsed_time(b) / 1000.0)
-    t = dist.max(statistics.median(times))
+
+    t = dist.max(graph_time(lambda: lay.step(c.q, fused=True), 20, 5, flush))
     by = cost.layer_bytes(w.seq_lens, w.Hq, w.Hkv, w.D, w.prefix, w.window, w.budget)
     peak, _ = hbm_peak()
     ach = by["sparse"] / t / 1e9
     # dense comparison on the same cache
     out = torch.empty_like(lay.out)
-
-    def dense():
-        csa.decode_full(d, c.q, c.k_cache, c.v_cache, c.page_table, c.seq_lens, out, lay.ws)
-
-    dense()
-    torch.cuda.synchronize()
-    dt = []
-    for i in range(15):
-        torch.sum(scrub, dim=0, out=sink)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        dense()
-        b.record()
-        torch.cuda.synchronize()
-        if i >= 3:
-            dt.append(a.elapsed_time(b) / 1000.0)
-    tdn = statistics.median(dt)
+    tdn = graph_time(lambda: csa.decode_full(d, c.q, c.k_cache, c.v_cache, c.page_table,
+                                             c.seq_lens, out, lay.ws), 10, 3, flush)
     return {"workload": w.name, "value": dist.world * w.B / t, "unit": UNIT,
             "us_per_layer_step": 1e6 * t, "algorithmic_bytes": by["sparse"],
             "achieved_gbs": ach, "frac_of_measured_peak": ach / peak,
             "frac_of_8tbs_nominal": ach / NOMINAL_HBM_GBS,
             "dense_us": 1e6 * tdn, "dense_gbs": by["dense"] / tdn / 1e9,
             "speedup_vs_dense": tdn / t,
-            "timing": "median of 25 graph replays, 256 MB L2 flush (read) between replays"}
+            "timing": "batches of 20 graph replays, each after a 256 MB L2 flush (read); the flush time subtracted; median of 3 batches"}
+
+
+def graph_time(fn, reps: int, warm: int, flush) -> float:
+    """CUDA-event time (s) of one graph replay of fn with L2 flushed (by a
+    read) before it: reps x (flush + replay) minus reps x flush, each between
+    one pair of events (a single replay is too short for the event clock's
+    2 us granularity on this system); the median of three such batches."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(warm):
+        flush()
+        g.replay()
+    torch.cuda.synchronize()
+
+    def batch(with_fn: bool) -> float:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            flush()
+            if with_fn:
+                g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / 1000.0
+
+    return statistics.median((batch(True) - batch(False)) / reps for _ in range(3))
+
+
+def run_sweep(args, dist: Dist):
+    """Sparse (csa_sparse_attention) against dense (csa_decode_full) decode on
+    the same cache, batch 4, 16 query / 4 kv heads, D 128, prefix 128, window
+    1024, at every length of the sweep grid and every budget; then the cost
+    model t = t0 + bytes / bw fitted to the sparse points by least squares."""
+    from long_context_decoding_b200 import csa
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the CUDA path has no CPU fallback)")
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    scrub = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MB
+    sink = torch.zeros((), device=dev)
+
+    def flush():
+        torch.sum(scrub, dim=0, out=sink)
+
+    points = []
+    for L in wl.SWEEP_GRID:
+        w = replace(wl.SWEEP, name=f"b4_h16x4_d128_ctx{L}", seq_lens=(L,) * 4)
+        c = wl.make_case(w, dev)
+        d = csa.make_dims(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.num_pages, w.max_pages)
+        lay = csa.Layer(d, c.k_cache, c.v_cache, c.page_table, c.seq_lens, w.prefix, w.window,
+                        0)
+        lay.rebuild_meta()
+        out = torch.empty_like(lay.out)
+        t_dense = graph_time(lambda: csa.decode_full(d, c.q, c.k_cache, c.v_cache,
+                                                       c.page_table, c.seq_lens, out, lay.ws),
+                               args.steps, args.warmup, flush)
+        for budget in wl.SWEEP_BUDGETS:
+            lay.budget = PS_TOKENS * w.max_pages if budget is None else budget
+            t = graph_time(lambda: lay.step(c.q, fused=True), args.steps, args.warmup, flush)
+            by = cost.layer_bytes(w.seq_lens, w.Hq, w.Hkv, w.D, w.prefix, w.window, budget)
+            points.append({"L": L, "budget": "all" if budget is None else budget,
+                           "sparse_us": 1e6 * t, "dense_us": 1e6 * t_dense,
+                           "speedup": t_dense / t, "sparse_bytes": by["sparse"],
+                           "dense_bytes": by["dense"], "sparse_gbs": by["sparse"] / t / 1e9})
+        assert csa.device_status(lay.ws) == 0
+        del c, lay, out
+        torch.cuda.empty_cache()
+    # cost model over the sparse points
+    x = [p["sparse_bytes"] for p in points]
+    y = [p["sparse_us"] * 1e-6 for p in points]
+    n = len(x)
+    mx, my = sum(x) / n, sum(y) / n
+    slope = sum((a - mx) * (b - my) for a, b in zip(x, y)) / sum((a - mx) ** 2 for a in x)
+    t0 = my - slope * mx
+    for p in points:
+        p["model_us"] = 1e6 * (t0 + slope * p["sparse_bytes"])
+    worst = max(abs(p["model_us"] - p["sparse_us"]) / p["sparse_us"] for p in points)
+    # a budget of "all" attends to every token: the same work as dense
+    beats = all(p["sparse_us"] < p["dense_us"] for p in points
+                if p["L"] >= 32768 and p["budget"] != "all")
+    all_ratio = min(p["dense_us"] / p["sparse_us"] for p in points if p["budget"] == "all")
+    line = {"metric": "sparse vs dense decode layer step over context length and budget",
+            "unit": "us", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "dtype": "bf16", "data": "synthetic (seeded Gaussian q/K/V, random page permutation)",
+            "config": {"workload": wl.SWEEP.name + " (uniform lengths)", "batch": 4,
+                       "q_heads": 16, "kv_heads": 4, "head_dim": 128, "prefix": 128,
+                       "window": 1024, "l2": "256 MB read between replays",
+                       "timing": "median of graph replays, CUDA events"},
+            "points": points,
+            "cost_model": {"t0_us": 1e6 * t0, "bw_gbs": 1.0 / slope / 1e9,
+                           "max_rel_err": worst, "form": "t = t0 + algorithmic bytes / bw"},
+            "sparse_faster_than_dense_for_all_L_ge_32k": beats,
+            "all_budget_min_speedup_vs_dense": all_ratio}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+PS_TOKENS = 16
 
 
 def main():
     args = parse_args()
     dist = Dist()
+    if args.sweep:
+        try:
+            run_sweep(args, dist)
+        finally:
+            dist.close()
+        return
     base = wl.CTX256K if args.workload == "ctx256k" else replace(wl.CTX64K, steps=0)
     if args.layers:
         base = replace(base, layers=args.layers)

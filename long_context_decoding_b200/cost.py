@@ -5,7 +5,8 @@ The decoding cost the pages' configuration search trades against accuracy
 memory-bound decode, the bytes a step must move.  Per (sequence, kv-head)
 unit with L tokens, prefix P, window W and budget:
 
-  * metadata of the top-k candidates: |C| pages x 4*D bytes (bf16 min + max);
+  * metadata of the candidates: |C| pages x 4*D bytes (bf16 min + max), when
+    there is a choice to make (0 < k < |C|; else no page needs a score);
   * K and V of the attended tokens:   |A| tokens x 4*D bytes;
   * q in and out: G*D*2 bytes each.
 
@@ -44,7 +45,9 @@ def unit_bytes(L: int, D: int, prefix: int, window: int, budget: Optional[int]) 
         n, mid = 0, 0
     k = n if budget is None else min(budget // PAGE, n)
     attended = Pe + We + min(mid, k * PAGE) if n else L
-    return UnitBytes(n, k, attended, n * 4 * D, attended * 4 * D)
+    # the metadata is read only when there is a choice to make (0 < k < |C|)
+    meta = n * 4 * D if 0 < k < n else 0
+    return UnitBytes(n, k, attended, meta, attended * 4 * D)
 
 
 def layer_bytes(seq_lens: Iterable[int], Hq: int, Hkv: int, D: int, prefix: int, window: int,

@@ -234,7 +234,9 @@ int csa_score_select(const csa_dims* d, const void* q, const void* meta,
     sp.keyrange = at<uint2>(workspace, w.keyrange);
     sp.flags = at<uint32_t>(workspace, w.flags);
     sp.s = s;
-    if (k_pages > 0 || scores_out) {
+    // scores are needed only where a unit has more candidates than it keeps
+    const long long n_max = (long long)s.MP - prefix / kPage - window / kPage;
+    if ((k_pages > 0 && k_pages < n_max) || scores_out) {
         rc = launch_status(launch_score(sp, st));
         if (rc != CSA_OK) {
             note_stream_call(stream, kCallOther);
@@ -362,7 +364,8 @@ int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
     sp.keyrange = at<uint2>(workspace, w.keyrange);
     sp.flags = at<uint32_t>(workspace, w.flags);
     sp.s = s;
-    if (k_pages > 0) {
+    const long long n_max = (long long)s.MP - prefix / kPage - window / kPage;
+    if (k_pages > 0 && k_pages < n_max) {      // else every unit keeps all its candidates
         rc = launch_status(launch_score(sp, st));
         if (rc != CSA_OK) return rc;
     }
@@ -388,7 +391,11 @@ int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
     dp.phase_floats = w.dec_slots * decode_record_floats(s);
     dp.s = s;
 
-    if (fused_eligible(s, prefix, window, k_pages)) {
+    // A budget that keeps every candidate of every unit attends to every
+    // token: the selection still reports all candidates, and the decode is
+    // the dense one (its work split suits a full sequence).
+    if (k_pages >= n_max) dp.dense = 1;
+    if (!dp.dense && fused_eligible(s, prefix, window, k_pages)) {
         FusedParams fp;
         fp.d = dp;
         fp.d.early = 1;
