@@ -189,13 +189,16 @@ class Clocks:
 
 
 # ---------------------------------------------------------------- CPU oracle
-def oracle_sample(w: wl.Workload, seconds: float, steps: int = 0, warmup: int = 0):
+def oracle_sample(w: wl.Workload, seconds: float, steps: int = 0, warmup: int = 0,
+                  threads: int = 0, dense: bool = False):
     """Time the CPU oracle on a bounded sample of workload ``w``: one
     sequence (all its kv-heads and query heads) of the first layer, full
-    length, one decode step (scores -> top-k -> attention) per iteration.
-    Returns (tokens/s per layer, iterations, seconds, threads)."""
+    length, one decode step (scores -> top-k -> attention; with dense, the
+    attention over every token) per iteration, on `threads` host threads (0:
+    every core the process may use).
+    Returns (tokens/s per layer, iterations, seconds, threads, sample)."""
     import oracle
-    threads = oracle.set_threads(len(os.sched_getaffinity(0)))
+    threads = oracle.set_threads(threads if threads > 0 else len(os.sched_getaffinity(0)))
     ws = replace(w, B=1, seq_lens=w.seq_lens[:1], layers=1, steps=0, spare_pages=0)
     c = wl.make_case(ws, "cpu", poison=False)
     window, budget = w.layer_window_budget(0)
@@ -205,8 +208,12 @@ def oracle_sample(w: wl.Workload, seconds: float, steps: int = 0, warmup: int = 
     scale = 1.0 / math.sqrt(ws.D)
 
     def one():
-        oracle.step(d, h["q"], h["k"], h["v"], h["pt"], h["sl"], ws.prefix, window, budget,
-                    max(1, budget // 16), scale)
+        if dense:
+            oracle.attend(d, h["q"], h["k"], h["v"], h["pt"], h["sl"], 0, 0, None, None, 1,
+                          scale, dense=True)
+        else:
+            oracle.step(d, h["q"], h["k"], h["v"], h["pt"], h["sl"], ws.prefix, window, budget,
+                        max(1, budget // 16), scale)
 
     for _ in range(warmup):
         one()
@@ -217,9 +224,10 @@ def oracle_sample(w: wl.Workload, seconds: float, steps: int = 0, warmup: int = 
         el = time.perf_counter() - t0
         if (steps and n >= steps) or (not steps and el >= seconds):
             break
+    what = "dense attention" if dense else "decode step"
     return n / el, n, el, threads, (f"1 of {w.B} sequences of layer 0 (window {window}, budget "
                                     f"{budget}) at {w.seq_lens[0]} tokens, all {w.Hkv} kv-heads "
-                                    f"and {w.Hq} query heads; one oracle decode step per "
+                                    f"and {w.Hq} query heads; one oracle {what} per "
                                     f"iteration, {n} iterations in {el:.1f} s")
 
 
@@ -456,8 +464,12 @@ def run_ours(args, dist: Dist, base: wl.Workload):
         # ---- CPU oracle on a bounded sample
         if not args.no_cpu_baseline and dist.rank == 0 and dist.world == 1:
             rate, n, el, threads, sample = oracle_sample(base, args.cpu_seconds)
+            r1, _, _, _, s1 = oracle_sample(base, args.cpu_seconds / 3, threads=1)
+            rd, _, _, td, sd = oracle_sample(base, args.cpu_seconds / 3, dense=True)
             line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads,
-                                    "kind": "oracle", "sample": sample}
+                                    "kind": "oracle", "sample": sample,
+                                    "one_core": {"value": r1, "cores": 1, "sample": s1},
+                                    "dense": {"value": rd, "cores": td, "sample": sd}}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -55,10 +55,11 @@
  *  - Kernels are launched with programmatic dependent launch, so a kernel
  *    may start while the previous kernel on the stream finishes.  Each call
  *    waits for the preceding work before it reads anything, with two
- *    exceptions.  (1) csa_score_select reads `page_table` and `seq_lens`
- *    early: those two must not come from the kernel launched just before the
- *    call if that kernel releases its dependents early (a host copy, an
- *    event, a plain kernel or a call of this library is fine).  (2) When the
+ *    exceptions.  (1) csa_meta_update, csa_score_select and
+ *    csa_sparse_attention read `page_table` and `seq_lens` early: those two
+ *    must not come from the kernel launched just before the call if that
+ *    kernel releases its dependents early (a host copy, an event, a plain
+ *    kernel or a call of this library is fine).  (2) When the
  *    previous call of this library on the same stream was csa_score_select,
  *    csa_decode / csa_decode_full stream the prefix and window pages while
  *    the selection kernel is still running: their `q`, `k_cache`,

@@ -39,12 +39,13 @@ __device__ __forceinline__ void fold(Pair& p, uint32_t v) {
 }
 
 // Append the new tokens of logical page `page` and refresh its min/max.
-__device__ void update_page(const MetaParams& p, int b, int g, int c, int L, int start, int page) {
-    const int Hkv = p.s.Hkv, D = p.s.D, MP = p.s.MP;
+// phys is the page's physical id (page_table[b][page]).
+__device__ void update_page(const MetaParams& p, int b, int g, int c, int L, int start, int page,
+                            int phys) {
+    const int Hkv = p.s.Hkv, D = p.s.D;
     const bool append = p.new_k != nullptr;
     const int t0 = page * kPage;
     const int t_end = t0 + kPage < L ? t0 + kPage : L;
-    const int phys = p.page_table[(size_t)b * MP + page];
     if (phys < 0 || phys >= p.s.NPG) {
         if (c == 0) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
         return;
@@ -94,23 +95,31 @@ __device__ void update_page(const MetaParams& p, int b, int g, int c, int L, int
 }
 
 __global__ void meta_update_kernel(MetaParams p) {
-    pdl_wait();
-    pdl_launch_dependents();
     const int u = blockIdx.x;
     const int Hkv = p.s.Hkv, D = p.s.D, MP = p.s.MP;
     const int b = u / Hkv, g = u % Hkv;
     const int c = threadIdx.x;                  // channel pair
+    // seq_lens and page_table are caller inputs, read before the dependency
+    // wait; the cache, the metadata and the new tokens only after it
     const int L = p.seq_lens[b];
     const bool append = p.new_k != nullptr;
-    if (L < 0 || L > MP * kPage || (append && L < p.n_new)) {
+    const bool bad_len = L < 0 || L > MP * kPage || (append && L < p.n_new);
+    const int start = bad_len ? 0 : (L - p.n_new > 0 ? L - p.n_new : 0);   // first new token
+    const int n_touched = bad_len || L == 0 ? 0 : (L - 1) / kPage - start / kPage + 1;
+    const int j0 = (int)blockIdx.y;
+    const int phys0 = j0 < n_touched ? p.page_table[(size_t)b * MP + start / kPage + j0] : -1;
+    pdl_wait();
+    pdl_launch_dependents();
+    if (bad_len) {
         if (c == 0 && blockIdx.y == 0) latch_flag(p.flags, CSA_DEVFLAG_BAD_SEQ_LEN);
         return;
     }
-    const int start = L - p.n_new > 0 ? L - p.n_new : 0;   // first new / rebuilt token
-    const int n_touched = (L - 1) / kPage - start / kPage + 1;
-    if (c >= D / 2 || L == 0) return;
-    for (int j = (int)blockIdx.y; j < n_touched; j += (int)gridDim.y)
-        update_page(p, b, g, c, L, start, start / kPage + j);
+    if (c >= D / 2) return;
+    for (int j = j0; j < n_touched; j += (int)gridDim.y) {
+        const int page = start / kPage + j;
+        const int phys = j == j0 ? phys0 : p.page_table[(size_t)b * MP + page];
+        update_page(p, b, g, c, L, start, page, phys);
+    }
 }
 
 }  // namespace
