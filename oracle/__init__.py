@@ -75,8 +75,17 @@ def _load():
         lib.oracle_select.argtypes = [P, P, P, I, I, I, I, P, P]
         lib.oracle_token_mask.argtypes = [P, P, I, I, P, P, I, I, P]
         lib.oracle_attend.argtypes = [P, P, P, P, P, P, I, I, P, P, I, I, ctypes.c_double, P, P]
+        lib.oracle_meta_fp8.argtypes = [P, P, P, P, P]
+        lib.oracle_scores_fp8.argtypes = [P, P, P, P, P, I, I, P]
+        lib.oracle_fp8_round.argtypes = [ctypes.c_double, I]
+        lib.oracle_fp8_round.restype = ctypes.c_double
+        lib.oracle_fp8_encode.argtypes = [ctypes.c_double]
+        lib.oracle_fp8_decode.argtypes = [I]
+        lib.oracle_fp8_decode.restype = ctypes.c_double
+        lib.oracle_fp8_row_exponent.argtypes = [ctypes.c_double]
         for f in (lib.oracle_set_threads, lib.oracle_meta, lib.oracle_scores, lib.oracle_select,
-                  lib.oracle_token_mask, lib.oracle_attend):
+                  lib.oracle_token_mask, lib.oracle_attend, lib.oracle_meta_fp8,
+                  lib.oracle_scores_fp8, lib.oracle_fp8_encode, lib.oracle_fp8_row_exponent):
             f.restype = I
         _lib = lib
     return _lib
@@ -186,3 +195,72 @@ def step(d: Dims, q, k_cache, v_cache, page_table, seq_lens, prefix: int, window
     out, lse = attend(d, q, k_cache, v_cache, page_table, seq_lens, prefix, window, sel, nsel,
                       max_sel, scale)
     return {"scores": sc, "sel": sel, "nsel": nsel, "out": out, "lse": lse}
+
+
+# ---------------------------------------------------------------- fp8 metadata
+# An optional lower-precision copy of the metadata (not a step of the pages'
+# method): per (physical page, kv-head) 2*D bytes of E4M3 -- min rounded down,
+# max rounded up after scaling by 2^-e -- and a 16-byte trailer holding e
+# (int32) and zeros.  See csa_oracle.c for the definition.
+def meta8_row_bytes(D: int) -> int:
+    return 2 * D + 16
+
+
+def fp8_round(y: float, up: bool) -> float:
+    """Largest (up=False) / smallest (up=True) E4M3 value <= / >= y (|y| <= 448)."""
+    return float(_load().oracle_fp8_round(float(y), 1 if up else 0))
+
+
+def fp8_encode(v: float) -> int:
+    return int(_load().oracle_fp8_encode(float(v)))
+
+
+def fp8_decode(x: int) -> float:
+    return float(_load().oracle_fp8_decode(int(x)))
+
+
+def fp8_row_exponent(a: float) -> int:
+    """Smallest e with a * 2^-e <= 448 (0 for a = 0)."""
+    return int(_load().oracle_fp8_row_exponent(float(a)))
+
+
+def meta_fp8(d: Dims, meta_bf16, page_table, seq_lens, meta8_init=None):
+    """fp8 copy of the (exact, bf16) metadata of every page reached by a valid
+    token.  Returns uint8 [num_pages][Hkv][2*D + 16]."""
+    lib = _load()
+    shape = (d.num_pages, d.Hkv, meta8_row_bytes(d.D))
+    out = np.zeros(shape, np.uint8) if meta8_init is None \
+        else np.array(meta8_init, dtype=np.uint8, copy=True)
+    m, mp = _c(meta_bf16, np.uint16)
+    pt, ptp = _c(page_table, np.int32)
+    sl, slp = _c(seq_lens, np.int32)
+    _check(lib.oracle_meta_fp8(d.arr(), mp, ptp, slp, out.ctypes.data_as(ctypes.c_void_p)),
+           "meta_fp8")
+    return out
+
+
+def scores_fp8(d: Dims, q, meta8, page_table, seq_lens, prefix: int, window: int):
+    """Quest scores from the fp8 metadata, float64 [B][Hkv][max_pages]; NaN off
+    the candidates."""
+    lib = _load()
+    out = np.empty((d.B, d.Hkv, d.max_pages), np.float64)
+    qq, qp = _c(q, np.uint16)
+    m8, m8p = _c(meta8, np.uint8)
+    pt, ptp = _c(page_table, np.int32)
+    sl, slp = _c(seq_lens, np.int32)
+    _check(lib.oracle_scores_fp8(d.arr(), qp, m8p, ptp, slp, int(prefix), int(window),
+                                 out.ctypes.data_as(ctypes.c_void_p)), "scores_fp8")
+    return out
+
+
+def step_fp8(d: Dims, q, k_cache, v_cache, page_table, seq_lens, prefix: int, window: int,
+             budget: int, max_sel: int, scale: float):
+    """One sparse decode step scored on the fp8 metadata (derived from the
+    exact metadata of the cache): scores -> top-k -> attention."""
+    m = meta(d, k_cache, page_table, seq_lens)
+    m8 = meta_fp8(d, m, page_table, seq_lens)
+    sc = scores_fp8(d, q, m8, page_table, seq_lens, prefix, window)
+    sel, nsel = select(d, sc, seq_lens, prefix, window, budget, max_sel)
+    out, lse = attend(d, q, k_cache, v_cache, page_table, seq_lens, prefix, window, sel, nsel,
+                      max_sel, scale)
+    return {"meta8": m8, "scores": sc, "sel": sel, "nsel": nsel, "out": out, "lse": lse}

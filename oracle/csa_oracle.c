@@ -398,3 +398,177 @@ int oracle_attend(const int *d, const uint16_t *q, const uint16_t *k_cache,
     free(mask);
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * fp8 page metadata (an optional variant of the scoring input, not a step of
+ * the pages' method: a lower-precision copy of the exact bf16 min/max that
+ * halves the bytes the scoring reads).  Each metadata row pair (the D minima
+ * and D maxima of one physical page and kv-head) is stored as
+ *     2*D bytes of OCP FP8 E4M3 (1 sign, 4 exponent bits with bias 7,
+ *     3 mantissa bits; largest finite value 448; subnormals k * 2^-9)
+ *     followed by a 16-byte trailer: int32 e, then 12 zero bytes,
+ * and encodes min * 2^-e rounded toward -inf and max * 2^-e rounded toward
+ * +inf, so the decoded box [2^e * min8, 2^e * max8] contains the exact one
+ * and the Quest bound computed from it is still an upper bound for every
+ * head.  e is the smallest integer with max_i |value_i| * 2^-e <= 448 over
+ * the row pair (0 for an all-zero row pair).  Zero is encoded as 0x00.
+ * ------------------------------------------------------------------------ */
+
+/* Largest (up = 0) or smallest (up = 1) E4M3 value <= (>=) y, |y| <= 448.  */
+static double fp8_round(double y, int up)
+{
+    if (y < 0.0)
+        return -fp8_round(-y, !up);
+    const double sub = ldexp(1.0, -9);     /* subnormal quantum             */
+    double quantum;
+    if (y < ldexp(1.0, -6)) {
+        quantum = sub;
+    } else {
+        int ex;
+        frexp(y, &ex);                     /* y = f * 2^ex, f in [0.5, 1)   */
+        quantum = ldexp(1.0, ex - 1 - 3);  /* 3 mantissa bits below 2^(ex-1) */
+    }
+    double k = up ? ceil(y / quantum) : floor(y / quantum);
+    return k * quantum;
+}
+
+/* E4M3 bit pattern of a value of the grid (zero -> 0x00).                  */
+static uint8_t fp8_encode(double v)
+{
+    if (v == 0.0)
+        return 0;
+    uint8_t s = v < 0.0 ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a < ldexp(1.0, -6))
+        return (uint8_t)(s | (uint8_t)(a / ldexp(1.0, -9)));
+    int ex;
+    frexp(a, &ex);
+    int E = ex - 1;                        /* a = m * 2^(E-3), m in [8, 15] */
+    int m = (int)(a / ldexp(1.0, E - 3));
+    return (uint8_t)(s | (uint8_t)((E + 7) << 3) | (uint8_t)(m - 8));
+}
+
+/* Value of an E4M3 bit pattern (0x7f / 0xff, NaN, never occur here).        */
+static double fp8_decode(uint8_t x)
+{
+    double sgn = (x & 0x80) ? -1.0 : 1.0;
+    int E = (x >> 3) & 0xF, m = x & 7;
+    if (E == 0)
+        return sgn * ldexp((double)m, -9);
+    return sgn * ldexp((double)(8 + m), E - 7 - 3);
+}
+
+/* Smallest e with a * 2^-e <= 448 (a = max |value| >= 0); 0 for a = 0.     */
+static int fp8_row_exponent(double a)
+{
+    if (a == 0.0)
+        return 0;
+    int ex;
+    double f = frexp(a, &ex);              /* a = f * 2^ex = (2f) * 2^(ex-1) */
+    int k = ex - 1;
+    return k - 8 + (2.0 * f > 1.75 ? 1 : 0);
+}
+
+/* Exported for the tests' pins.                                             */
+double oracle_fp8_round(double y, int up) { return fp8_round(y, up); }
+int oracle_fp8_encode(double v) { return fp8_encode(v); }
+double oracle_fp8_decode(int x) { return fp8_decode((uint8_t)x); }
+int oracle_fp8_row_exponent(double a) { return fp8_row_exponent(a); }
+
+/* fp8 copy of the metadata of every physical page that a sequence reaches
+ * through a valid token.  meta: [num_pages][Hkv][2][D] bf16 (exact min/max);
+ * meta8: [num_pages][Hkv][2*D + 16] bytes; untouched pages keep their bytes. */
+int oracle_meta_fp8(const int *d, const uint16_t *meta, const int32_t *page_table,
+                    const int32_t *seq_lens, uint8_t *meta8)
+{
+    if (!dims_ok(d))
+        return ORACLE_EINVAL;
+    const int B = d[0], Hkv = d[2], D = d[3], ps = d[4], MP = d[5], NPG = d[6];
+    const size_t row = (size_t)2 * D + 16;
+    for (int b = 0; b < B; ++b) {
+        int L = seq_lens[b];
+        if (L < 0 || L > MP * ps)
+            return ORACLE_EINVAL;
+        int np = (L + ps - 1) / ps;
+        for (int p = 0; p < np; ++p) {
+            int phys = page_table[(size_t)b * MP + p];
+            if (phys < 0 || phys >= NPG)
+                return ORACLE_EINVAL;
+            for (int g = 0; g < Hkv; ++g) {
+                const uint16_t *mn = meta + (((size_t)phys * Hkv + g) * 2 + 0) * D;
+                const uint16_t *mx = meta + (((size_t)phys * Hkv + g) * 2 + 1) * D;
+                uint8_t *out = meta8 + ((size_t)phys * Hkv + g) * row;
+                double amax = 0.0;
+                for (int i = 0; i < D; ++i) {
+                    if (fabs(bf(mn[i])) > amax)
+                        amax = fabs(bf(mn[i]));
+                    if (fabs(bf(mx[i])) > amax)
+                        amax = fabs(bf(mx[i]));
+                }
+                int e = fp8_row_exponent(amax);
+                for (int i = 0; i < D; ++i) {
+                    out[i] = fp8_encode(fp8_round(ldexp(bf(mn[i]), -e), 0));
+                    out[D + i] = fp8_encode(fp8_round(ldexp(bf(mx[i]), -e), 1));
+                }
+                int32_t e32 = e;
+                memcpy(out + 2 * D, &e32, 4);
+                memset(out + 2 * D + 4, 0, 12);
+            }
+        }
+    }
+    return 0;
+}
+
+/* Quest scores from fp8 metadata (the stored box, decoded and scaled by 2^e):
+ * same candidates, layout and NaN convention as oracle_scores.              */
+int oracle_scores_fp8(const int *d, const uint16_t *q, const uint8_t *meta8,
+                      const int32_t *page_table, const int32_t *seq_lens, int prefix,
+                      int window, double *scores)
+{
+    if (!dims_ok(d) || prefix < 0 || window < 0)
+        return ORACLE_EINVAL;
+    const int B = d[0], Hq = d[1], Hkv = d[2], D = d[3], ps = d[4], MP = d[5],
+              NPG = d[6];
+    const int G = Hq / Hkv;
+    const size_t row = (size_t)2 * D + 16;
+    for (int b = 0; b < B; ++b) {
+        if (seq_lens[b] < 0 || seq_lens[b] > MP * ps)
+            return ORACLE_EINVAL;
+        int np = (seq_lens[b] + ps - 1) / ps;
+        for (int p = 0; p < np; ++p) {
+            int phys = page_table[(size_t)b * MP + p];
+            if (phys < 0 || phys >= NPG)
+                return ORACLE_EINVAL;
+        }
+    }
+    for (size_t i = 0; i < (size_t)B * Hkv * MP; ++i)
+        scores[i] = NAN;
+    int units = B * Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int u = 0; u < units; ++u) {
+        int b = u / Hkv, g = u % Hkv;
+        int Pe, We, c_lo, c_hi;
+        ranges(seq_lens[b], prefix, window, ps, &Pe, &We, &c_lo, &c_hi);
+        for (int p = c_lo; p < c_hi; ++p) {
+            int phys = page_table[(size_t)b * MP + p];
+            const uint8_t *r = meta8 + ((size_t)phys * Hkv + g) * row;
+            int32_t e;
+            memcpy(&e, r + 2 * D, 4);
+            double best = -INFINITY;
+            for (int j = 0; j < G; ++j) {
+                const uint16_t *qh = q + ((size_t)b * Hq + (size_t)g * G + j) * D;
+                double s = 0.0;
+                for (int i = 0; i < D; ++i) {
+                    double qi = bf(qh[i]);
+                    double lo = ldexp(fp8_decode(r[i]), e), hi = ldexp(fp8_decode(r[D + i]), e);
+                    double a = qi * hi, c = qi * lo;
+                    s += a > c ? a : c;
+                }
+                if (s > best)
+                    best = s;
+            }
+            scores[((size_t)b * Hkv + g) * MP + p] = best;
+        }
+    }
+    return 0;
+}
