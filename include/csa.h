@@ -217,6 +217,40 @@ int csa_sparse_attention(const csa_dims *d, const void *q, const void *k_cache,
                          float *lse, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * fp8 metadata (an option; the pages specify no metadata precision, and the
+ * entry points above use the exact bf16 min/max).  meta8 is a lower-precision
+ * copy of meta that the scoring reads instead, moving about half the bytes:
+ *   meta8  uint8 [num_pages][Hkv][2*D + 16]
+ * per (physical page, kv-head): D bytes of E4M3 (OCP FP8: bias 7, 3 mantissa
+ * bits, largest value 448) for min * 2^-e rounded toward -inf, D bytes for
+ * max * 2^-e rounded toward +inf, then a 16-byte trailer {int32 e, 0, 0, 0}.
+ * e is the smallest integer with max |value| * 2^-e <= 448 over the two rows
+ * (0 when they are all zero).  The decoded box [2^e min8, 2^e max8] contains
+ * the exact one, so the Quest score from it is still an upper bound for every
+ * head; it may be looser, so the selection can differ from the bf16 one.
+ *
+ * csa_meta_update_fp8: csa_meta_update, and the fp8 copy of every page whose
+ *   metadata it writes (meta stays the exact master copy).
+ * csa_score_select_fp8 / csa_sparse_attention_fp8: csa_score_select /
+ *   csa_sparse_attention with the scores computed from meta8.
+ */
+int csa_meta_update_fp8(const csa_dims *d, void *k_cache, void *v_cache, void *meta,
+                        void *meta8, const int32_t *page_table, const int32_t *seq_lens,
+                        const void *new_k, const void *new_v, int n_new,
+                        void *workspace, size_t workspace_bytes, void *stream);
+int csa_score_select_fp8(const csa_dims *d, const void *q, const void *meta8,
+                         const int32_t *page_table, const int32_t *seq_lens,
+                         int prefix, int window, int budget_tokens,
+                         int32_t *sel_pages, int32_t *n_sel, float *scores_out,
+                         void *workspace, size_t workspace_bytes, void *stream);
+int csa_sparse_attention_fp8(const csa_dims *d, const void *q, const void *k_cache,
+                             const void *v_cache, const void *meta8,
+                             const int32_t *page_table, const int32_t *seq_lens,
+                             int prefix, int window, int budget_tokens, float scale,
+                             int32_t *sel_pages, int32_t *n_sel, void *out, float *lse,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * csa_decode for callers that cannot allocate device memory.  The paper has
  * no counterpart to this entry point; it exists for deployment: a plugin
  * hosted inside another runtime that owns every device buffer, or a server

@@ -26,7 +26,8 @@ DEVFLAG_TIMEOUT = 8
 
 EXPORTS = ("csa_version", "csa_status_string", "csa_workspace_size", "csa_workspace_init",
            "csa_meta_update", "csa_score_select", "csa_decode", "csa_decode_full",
-           "csa_get_device_status", "csa_decode_noalloc", "csa_sparse_attention")
+           "csa_get_device_status", "csa_decode_noalloc", "csa_sparse_attention",
+           "csa_meta_update_fp8", "csa_score_select_fp8", "csa_sparse_attention_fp8")
 
 
 class CsaError(RuntimeError):
@@ -77,8 +78,13 @@ def lib() -> ctypes.CDLL:
         L.csa_get_device_status.argtypes = [P, P, ctypes.POINTER(I)]
         L.csa_sparse_attention.argtypes = [D, P, P, P, P, P, P, I, I, I, ctypes.c_float, P, P, P,
                                            P, P, Z, P]
+        L.csa_meta_update_fp8.argtypes = [D, P, P, P, P, P, P, P, P, I, P, Z, P]
+        L.csa_score_select_fp8.argtypes = [D, P, P, P, P, I, I, I, P, P, P, P, Z, P]
+        L.csa_sparse_attention_fp8.argtypes = [D, P, P, P, P, P, P, I, I, I, ctypes.c_float, P,
+                                               P, P, P, P, Z, P]
         for f in ("csa_workspace_init", "csa_meta_update", "csa_score_select", "csa_decode",
-                  "csa_decode_full", "csa_get_device_status", "csa_sparse_attention"):
+                  "csa_decode_full", "csa_get_device_status", "csa_sparse_attention",
+                  "csa_meta_update_fp8", "csa_score_select_fp8", "csa_sparse_attention_fp8"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -177,6 +183,54 @@ def sparse_attention(d: Dims, q, k_cache, v_cache, meta, page_table, seq_lens, p
         _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def meta8_row_bytes(D: int) -> int:
+    """Bytes of one (page, kv-head) row of the fp8 metadata copy."""
+    return 2 * D + 16
+
+
+def new_meta8(d: Dims, device="cuda") -> torch.Tensor:
+    """fp8 metadata copy, uint8 [num_pages][Hkv][2*D + 16]."""
+    return torch.zeros((d.num_pages, d.Hkv, meta8_row_bytes(d.D)), dtype=torch.uint8,
+                       device=device)
+
+
+def meta_update_fp8(d: Dims, k_cache, v_cache, meta, meta8, page_table, seq_lens, new_k, new_v,
+                    n_new: int, ws, stream=None):
+    """csa_meta_update that also keeps the fp8 copy meta8 current."""
+    bf = torch.bfloat16
+    _check("csa_meta_update_fp8", lib().csa_meta_update_fp8(
+        ctypes.byref(d), _ptr(k_cache, bf, "k_cache"), _ptr(v_cache, bf, "v_cache"),
+        _ptr(meta, bf, "meta"), _ptr(meta8, torch.uint8, "meta8"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        _ptr(new_k, bf, "new_k"), _ptr(new_v, bf, "new_v"), int(n_new), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def score_select_fp8(d: Dims, q, meta8, page_table, seq_lens, prefix: int, window: int,
+                     budget: int, sel, n_sel, ws, scores_out=None, stream=None):
+    """csa_score_select with the scores from the fp8 metadata copy."""
+    _check("csa_score_select_fp8", lib().csa_score_select_fp8(
+        ctypes.byref(d), _ptr(q, torch.bfloat16, "q"), _ptr(meta8, torch.uint8, "meta8"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        int(prefix), int(window), int(budget), _ptr(sel, torch.int32, "sel"),
+        _ptr(n_sel, torch.int32, "n_sel"), _ptr(scores_out, torch.float32, "scores_out"),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def sparse_attention_fp8(d: Dims, q, k_cache, v_cache, meta8, page_table, seq_lens,
+                         prefix: int, window: int, budget: int, sel, n_sel, out, ws, lse=None,
+                         scale: float = 0.0, stream=None):
+    """csa_sparse_attention with the scores from the fp8 metadata copy."""
+    bf = torch.bfloat16
+    _check("csa_sparse_attention_fp8", lib().csa_sparse_attention_fp8(
+        ctypes.byref(d), _ptr(q, bf, "q"), _ptr(k_cache, bf, "k_cache"),
+        _ptr(v_cache, bf, "v_cache"), _ptr(meta8, torch.uint8, "meta8"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        int(prefix), int(window), int(budget), float(scale), _ptr(sel, torch.int32, "sel"),
+        _ptr(n_sel, torch.int32, "n_sel"), _ptr(out, bf, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
 def decode_full(d: Dims, q, k_cache, v_cache, page_table, seq_lens, out, ws, lse=None,
                 scale: float = 0.0, stream=None):
     """Dense decode over every valid token (the unmodified layer)."""
@@ -226,7 +280,7 @@ class Layer:
     C ABI: append + metadata update, score + select, sparse decode."""
 
     def __init__(self, d: Dims, k_cache, v_cache, page_table, seq_lens, prefix: int, window: int,
-                 budget: int, meta=None, ws=None):
+                 budget: int, meta=None, ws=None, fp8: bool = False):
         self.d = d
         dev = k_cache.device
         self.k_cache, self.v_cache = k_cache, v_cache
@@ -235,6 +289,8 @@ class Layer:
         self.meta = meta if meta is not None else torch.zeros(
             (d.num_pages, d.Hkv, 2, d.D), dtype=torch.bfloat16, device=dev)
         self.ws = ws if ws is not None else new_workspace(d, dev)
+        # fp8: also keep the fp8 metadata copy and score from it
+        self.meta8 = new_meta8(d, dev) if fp8 else None
         self.sel = torch.zeros((d.B, d.Hkv, d.max_sel), dtype=torch.int32, device=dev)
         self.n_sel = torch.zeros((d.B, d.Hkv), dtype=torch.int32, device=dev)
         self.out = torch.empty((d.B, d.Hq, d.D), dtype=torch.bfloat16, device=dev)
@@ -242,6 +298,10 @@ class Layer:
 
     def rebuild_meta(self, stream=None):
         n = self.d.max_pages_per_seq * PAGE
+        if self.meta8 is not None:
+            meta_update_fp8(self.d, self.k_cache, self.v_cache, self.meta, self.meta8,
+                            self.page_table, self.seq_lens, None, None, n, self.ws, stream)
+            return
         meta_update(self.d, self.k_cache, self.v_cache, self.meta, self.page_table, self.seq_lens,
                     None, None, n, self.ws, stream)
 
@@ -249,6 +309,24 @@ class Layer:
         """One decode step.  With new_k/new_v ([B][1][Hkv][D]) the token is
         appended first; seq_lens must already count it.  fused=True runs
         scoring, selection and decode as one csa_sparse_attention call."""
+        if self.meta8 is not None:
+            if new_k is not None:
+                meta_update_fp8(self.d, self.k_cache, self.v_cache, self.meta, self.meta8,
+                                self.page_table, self.seq_lens, new_k, new_v, new_k.shape[1],
+                                self.ws, stream)
+            if fused:
+                sparse_attention_fp8(self.d, q, self.k_cache, self.v_cache, self.meta8,
+                                     self.page_table, self.seq_lens, self.prefix, self.window,
+                                     self.budget, self.sel, self.n_sel, self.out, self.ws,
+                                     self.lse, stream=stream)
+            else:
+                score_select_fp8(self.d, q, self.meta8, self.page_table, self.seq_lens,
+                                 self.prefix, self.window, self.budget, self.sel, self.n_sel,
+                                 self.ws, stream=stream)
+                decode(self.d, q, self.k_cache, self.v_cache, self.page_table, self.seq_lens,
+                       self.sel, self.n_sel, self.prefix, self.window, self.out, self.ws,
+                       self.lse, stream=stream)
+            return self.out
         if new_k is not None:
             meta_update(self.d, self.k_cache, self.v_cache, self.meta, self.page_table,
                         self.seq_lens, new_k, new_v, new_k.shape[1], self.ws, stream)

@@ -164,10 +164,10 @@ int csa_workspace_init(void* workspace, size_t bytes, void* stream) {
     return launch_status(cudaMemsetAsync(workspace, 0, bytes, (cudaStream_t)stream));
 }
 
-int csa_meta_update(const csa_dims* d, void* k_cache, void* v_cache, void* meta,
-                    const int32_t* page_table, const int32_t* seq_lens, const void* new_k,
-                    const void* new_v, int n_new, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+static int meta_update_common(const csa_dims* d, void* k_cache, void* v_cache, void* meta,
+                              void* meta8, const int32_t* page_table, const int32_t* seq_lens,
+                              const void* new_k, const void* new_v, int n_new, void* workspace,
+                              size_t workspace_bytes, void* stream) {
     Shape s;
     int rc = check_dims(d, &s);
     if (rc != CSA_OK) return rc;
@@ -194,6 +194,7 @@ int csa_meta_update(const csa_dims* d, void* k_cache, void* v_cache, void* meta,
     p.seq_lens = seq_lens;
     p.new_k = static_cast<const uint16_t*>(new_k);
     p.new_v = static_cast<const uint16_t*>(new_v);
+    p.meta8 = static_cast<uint8_t*>(meta8);
     p.n_new = n_new;
     p.flags = at<uint32_t>(workspace, w.flags);
     p.s = s;
@@ -201,15 +202,20 @@ int csa_meta_update(const csa_dims* d, void* k_cache, void* v_cache, void* meta,
     return launch_status(launch_meta_update(p, (cudaStream_t)stream));
 }
 
-int csa_score_select(const csa_dims* d, const void* q, const void* meta,
-                     const int32_t* page_table, const int32_t* seq_lens, int prefix, int window,
-                     int budget_tokens, int32_t* sel_pages, int32_t* n_sel, float* scores_out,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+static int score_select_common(const csa_dims* d, const void* q, const void* meta,
+                               const void* meta8, const int32_t* page_table,
+                               const int32_t* seq_lens, int prefix, int window, int budget_tokens,
+                               int32_t* sel_pages, int32_t* n_sel, float* scores_out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
     Shape s;
     int rc = check_dims(d, &s);
     if (rc != CSA_OK) return rc;
     CSA_REQUIRE(q);
-    CSA_REQUIRE(meta);
+    if (meta8) {
+        CSA_REQUIRE(meta8);
+    } else {
+        CSA_REQUIRE(meta);
+    }
     CSA_REQUIRE(page_table);
     CSA_REQUIRE(seq_lens);
     CSA_REQUIRE(sel_pages);
@@ -231,6 +237,7 @@ int csa_score_select(const csa_dims* d, const void* q, const void* meta,
     sp.window = window;
     sp.scores_ws = at<float>(workspace, w.scores);
     sp.scores_out = scores_out;
+    sp.meta8 = static_cast<const uint8_t*>(meta8);
     sp.keyrange = at<uint2>(workspace, w.keyrange);
     sp.flags = at<uint32_t>(workspace, w.flags);
     sp.s = s;
@@ -324,18 +331,23 @@ int csa_decode_full(const csa_dims* d, const void* q, const void* k_cache, const
                          scale, out, lse, workspace, workspace_bytes, stream);
 }
 
-int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
-                         const void* v_cache, const void* meta, const int32_t* page_table,
-                         const int32_t* seq_lens, int prefix, int window, int budget_tokens,
-                         float scale, int32_t* sel_pages, int32_t* n_sel, void* out, float* lse,
-                         void* workspace, size_t workspace_bytes, void* stream) {
+static int sparse_attention_common(const csa_dims* d, const void* q, const void* k_cache,
+                                   const void* v_cache, const void* meta, const void* meta8,
+                                   const int32_t* page_table, const int32_t* seq_lens, int prefix,
+                                   int window, int budget_tokens, float scale,
+                                   int32_t* sel_pages, int32_t* n_sel, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
     Shape s;
     int rc = check_dims(d, &s);
     if (rc != CSA_OK) return rc;
     CSA_REQUIRE(q);
     CSA_REQUIRE(k_cache);
     CSA_REQUIRE(v_cache);
-    CSA_REQUIRE(meta);
+    if (meta8) {
+        CSA_REQUIRE(meta8);
+    } else {
+        CSA_REQUIRE(meta);
+    }
     CSA_REQUIRE(page_table);
     CSA_REQUIRE(seq_lens);
     CSA_REQUIRE(sel_pages);
@@ -361,6 +373,7 @@ int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
     sp.window = window;
     sp.scores_ws = at<float>(workspace, w.scores);
     sp.scores_out = nullptr;
+    sp.meta8 = static_cast<const uint8_t*>(meta8);
     sp.keyrange = at<uint2>(workspace, w.keyrange);
     sp.flags = at<uint32_t>(workspace, w.flags);
     sp.s = s;
@@ -423,6 +436,64 @@ int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
     if (rc != CSA_OK) return rc;
     dp.early = 1;   // our own scoring and selection kernels are the ones ahead
     return launch_status(launch_decode(dp, st));
+}
+
+int csa_meta_update(const csa_dims* d, void* k_cache, void* v_cache, void* meta,
+                    const int32_t* page_table, const int32_t* seq_lens, const void* new_k,
+                    const void* new_v, int n_new, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+    return meta_update_common(d, k_cache, v_cache, meta, nullptr, page_table, seq_lens, new_k,
+                              new_v, n_new, workspace, workspace_bytes, stream);
+}
+
+int csa_meta_update_fp8(const csa_dims* d, void* k_cache, void* v_cache, void* meta,
+                        void* meta8, const int32_t* page_table, const int32_t* seq_lens,
+                        const void* new_k, const void* new_v, int n_new, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+    CSA_REQUIRE(meta8);
+    return meta_update_common(d, k_cache, v_cache, meta, meta8, page_table, seq_lens, new_k,
+                              new_v, n_new, workspace, workspace_bytes, stream);
+}
+
+int csa_score_select(const csa_dims* d, const void* q, const void* meta,
+                     const int32_t* page_table, const int32_t* seq_lens, int prefix, int window,
+                     int budget_tokens, int32_t* sel_pages, int32_t* n_sel, float* scores_out,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+    return score_select_common(d, q, meta, nullptr, page_table, seq_lens, prefix, window,
+                               budget_tokens, sel_pages, n_sel, scores_out, workspace,
+                               workspace_bytes, stream);
+}
+
+int csa_score_select_fp8(const csa_dims* d, const void* q, const void* meta8,
+                         const int32_t* page_table, const int32_t* seq_lens, int prefix,
+                         int window, int budget_tokens, int32_t* sel_pages, int32_t* n_sel,
+                         float* scores_out, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    CSA_REQUIRE(meta8);
+    return score_select_common(d, q, nullptr, meta8, page_table, seq_lens, prefix, window,
+                               budget_tokens, sel_pages, n_sel, scores_out, workspace,
+                               workspace_bytes, stream);
+}
+
+int csa_sparse_attention(const csa_dims* d, const void* q, const void* k_cache,
+                         const void* v_cache, const void* meta, const int32_t* page_table,
+                         const int32_t* seq_lens, int prefix, int window, int budget_tokens,
+                         float scale, int32_t* sel_pages, int32_t* n_sel, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    return sparse_attention_common(d, q, k_cache, v_cache, meta, nullptr, page_table, seq_lens,
+                                   prefix, window, budget_tokens, scale, sel_pages, n_sel, out,
+                                   lse, workspace, workspace_bytes, stream);
+}
+
+int csa_sparse_attention_fp8(const csa_dims* d, const void* q, const void* k_cache,
+                             const void* v_cache, const void* meta8, const int32_t* page_table,
+                             const int32_t* seq_lens, int prefix, int window, int budget_tokens,
+                             float scale, int32_t* sel_pages, int32_t* n_sel, void* out,
+                             float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    CSA_REQUIRE(meta8);
+    return sparse_attention_common(d, q, k_cache, v_cache, nullptr, meta8, page_table, seq_lens,
+                                   prefix, window, budget_tokens, scale, sel_pages, n_sel, out,
+                                   lse, workspace, workspace_bytes, stream);
 }
 
 int csa_get_device_status(void* workspace, void* stream, int* flags_out) {

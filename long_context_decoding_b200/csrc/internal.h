@@ -32,6 +32,7 @@ struct MetaParams {
     const int32_t* seq_lens;
     const uint16_t* new_k;   // nullable (rebuild)
     const uint16_t* new_v;
+    uint8_t* meta8;          // nullable: fp8 copy [num_pages][Hkv][2D + 16] to keep current
     int n_new;
     uint32_t* flags;
     Shape s;
@@ -47,6 +48,7 @@ struct ScoreParams {
     int prefix, window;
     float* scores_ws;       // [B][Hkv][MP]
     float* scores_out;      // nullable
+    const uint8_t* meta8;   // non-null: score from the fp8 copy instead of meta
     uint2* keyrange;        // [units] merged with atomicMax: ~min key, max key
     uint32_t* flags;
     Shape s;

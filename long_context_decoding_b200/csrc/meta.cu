@@ -38,6 +38,84 @@ __device__ __forceinline__ void fold(Pair& p, uint32_t v) {
     p.hi = sel_half(p.hi, v, 1, v1 > bf16_hi(p.hi));
 }
 
+// ---------------------------------------------------------------- fp8 copy
+// The optional fp8 copy of a metadata row pair: 2*D bytes of E4M3 (OCP FP8:
+// bias 7, 3 mantissa bits, largest value 448, subnormals k * 2^-9) holding
+// min * 2^-e rounded toward -inf and max * 2^-e rounded toward +inf, then a
+// 16-byte trailer {e, 0, 0, 0} (int32).  e is the smallest integer with
+// max |value| * 2^-e <= 448 over the row pair (0 when it is all zero), so
+// the decoded box contains the exact one and the Quest bound stays an upper
+// bound.  All steps below are exact in fp32: scaling by powers of two and
+// floor/ceil of quotients by powers of two.
+
+// Largest (up = false) / smallest (up = true) E4M3 value <= / >= y, |y| <= 448.
+__device__ float fp8_round(float y, bool up) {
+    const bool neg = y < 0.f;
+    if (neg) {
+        y = -y;
+        up = !up;
+    }
+    float quantum = 0.001953125f;                    // 2^-9 below 2^-6
+    if (y >= 0.015625f) {
+        int ex;
+        frexpf(y, &ex);                              // y in [2^(ex-1), 2^ex)
+        quantum = ldexpf(1.f, ex - 4);               // 3 mantissa bits
+    }
+    const float k = up ? ceilf(y / quantum) : floorf(y / quantum);
+    const float r = k * quantum;
+    return neg ? -r : r;
+}
+
+// E4M3 bits of a value on the grid; zero is 0x00.
+__device__ uint32_t fp8_encode(float v) {
+    if (v == 0.f) return 0u;
+    const uint32_t s = v < 0.f ? 0x80u : 0u;
+    const float a = fabsf(v);
+    if (a < 0.015625f) return s | (uint32_t)(a * 512.f);
+    int ex;
+    frexpf(a, &ex);
+    const int E = ex - 1;
+    const int m = (int)ldexpf(a, 3 - E);             // 8 .. 15
+    return s | ((uint32_t)(E + 7) << 3) | (uint32_t)(m - 8);
+}
+
+__device__ uint32_t fp8_outward(float x, int e, bool up) {
+    float y = ldexpf(x, -e);
+    // below 2^-10 only the sign decides (and fp32 may have underflowed)
+    if (x != 0.f && fabsf(y) < 0.0009765625f) y = copysignf(0.0009765625f, x);
+    return fp8_encode(fp8_round(y, up));
+}
+
+// Called by all D/2 threads of the CTA (thread c owns channels 2c, 2c+1).
+__device__ void write_fp8_row(const MetaParams& p, int phys, int g, int c, const Pair& acc) {
+    __shared__ uint32_t s_max[4];
+    const int D = p.s.D;
+    const int warp = c >> 5, lane = c & 31;
+    const float mn0 = bf16_lo(acc.lo), mn1 = bf16_hi(acc.lo);
+    const float mx0 = bf16_lo(acc.hi), mx1 = bf16_hi(acc.hi);
+    const float a = fmaxf(fmaxf(fabsf(mn0), fabsf(mn1)), fmaxf(fabsf(mx0), fabsf(mx1)));
+    // non-negative floats order like their bit patterns
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(a));
+    if (lane == 0) s_max[warp] = wmax;
+    __syncthreads();
+    uint32_t amax_bits = 0;
+    for (int w = 0; w < (D / 2 + 31) / 32; ++w) amax_bits = max(amax_bits, s_max[w]);
+    __syncthreads();            // s_max is reused by the next page of this CTA
+    const float amax = __uint_as_float(amax_bits);
+    int e = 0;
+    if (amax > 0.f) {
+        int ex;
+        const float f = frexpf(amax, &ex);           // amax = (2f) * 2^(ex-1)
+        e = ex - 1 - 8 + (2.f * f > 1.75f ? 1 : 0);
+    }
+    uint8_t* row = p.meta8 + ((size_t)phys * p.s.Hkv + g) * (size_t)(2 * D + 16);
+    const uint32_t lo = fp8_outward(mn0, e, false) | (fp8_outward(mn1, e, false) << 8);
+    const uint32_t hi = fp8_outward(mx0, e, true) | (fp8_outward(mx1, e, true) << 8);
+    reinterpret_cast<uint16_t*>(row)[c] = (uint16_t)lo;
+    reinterpret_cast<uint16_t*>(row + D)[c] = (uint16_t)hi;
+    if (c == 0) *reinterpret_cast<int4*>(row + 2 * D) = make_int4(e, 0, 0, 0);
+}
+
 // Append the new tokens of logical page `page` and refresh its min/max.
 // phys is the page's physical id (page_table[b][page]).
 __device__ void update_page(const MetaParams& p, int b, int g, int c, int L, int start, int page,
@@ -92,6 +170,7 @@ __device__ void update_page(const MetaParams& p, int b, int g, int c, int L, int
     }
     mt[c] = acc.lo;
     mt[W + c] = acc.hi;
+    if (p.meta8) write_fp8_row(p, phys, g, c, acc);
 }
 
 __global__ void meta_update_kernel(MetaParams p) {

@@ -124,8 +124,42 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     return v;
 }
 
-template <int D, int NB>
-__global__ void __launch_bounds__(ScoreCfg<D, NB>::kThreads)
+// 4-byte load that does not allocate in L1 (the fp8 row exponent).
+__device__ __forceinline__ int ld_stream_s32(const void* p) {
+    int v;
+    asm volatile("ld.global.nc.L1::no_allocate.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// Two E4M3 values (bytes 0 and 1 of w) -> f16x2, exactly (hardware cvt).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h2)
+        : "r"(w));
+    return h2;
+}
+// 8 E4M3 channels -> 8 f16 channels in the order of a 16-byte chunk.
+__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint32_t lo, uint32_t hi) {
+    return make_uint4(e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi),
+                      e4m3x2_to_f16x2(hi >> 16));
+}
+// bf16x2 -> f16x2 (exact for |x| in [2^-17, 65504]; larger values saturate).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(bf16_hi(w)), "f"(bf16_lo(w)));
+    return r;
+}
+
+// F8: the metadata is the fp8 copy (rows of 2D E4M3 bytes + a 16-byte trailer
+// whose first int32 is the row's exponent e): 16 channels per 16-byte load,
+// converted by the hardware to f16 (one instruction per two channels; the
+// three-step route to bf16 made the conversions the bottleneck), multiplied
+// with q in f16 on the tensor cores (products exact in fp32; q is exact in
+// f16 for |q| >= 2^-17), and the row's sums scaled by 2^e.
+template <int D, int NB, bool F8>
+__global__ void __launch_bounds__(ScoreCfg<D, NB>::kThreads,
+                                  ((NB == 1 && !(F8 && D == 256)) || D == 64) ? 2 : 1)
 score_kernel(ScoreParams p) {
     using C = ScoreCfg<D, NB>;
     extern __shared__ __align__(16) int smem_i[];
@@ -197,105 +231,259 @@ score_kernel(ScoreParams p) {
     const int gq = lane >> 2, tq = lane & 3;
     uint32_t qf[C::kKPairs][NB][4];          // B fragments of [q- | q+] for the current unit
     int cur_unit = -1;
-    walk.start(s, e);
-    TileInfo t;
     int kr_unit = -1;                        // key range of this warp's current unit
     uint32_t kr_nmin = 0u, kr_max = 0u;
-    for (int j = 0; walk.next(t); ++j) {
-        if (j % C::kWarps != warp) continue;
-        const int b = t.unit / Hkv, g = t.unit % Hkv;
-        const int x0 = walk.x - t.count - s;           // slice index of row 0
-        // rows g and g+8 of the tile (clamped inside the tile; extra rows are dropped)
-        const int r0 = gq < t.count ? gq : t.count - 1;
-        const int r8 = gq + 8 < t.count ? gq + 8 : t.count - 1;
-        const int p0 = pt[x0 + r0], p8 = pt[x0 + r8];
-        const bool ok0 = p0 >= 0 && p0 < p.s.NPG, ok8 = p8 >= 0 && p8 < p.s.NPG;
-        const char* row0 = reinterpret_cast<const char*>(
-            p.meta + ((size_t)(ok0 ? p0 : 0) * Hkv + g) * 2 * D) + 16 * tq;
-        const char* row8 = reinterpret_cast<const char*>(
-            p.meta + ((size_t)(ok8 ? p8 : 0) * Hkv + g) * 2 * D) + 16 * tq;
-        uint4 xa[C::kKPairs], xb[C::kKPairs];
+    if constexpr (F8) {
+        // registers of one tile: rows g and g+8 of the fp8 copy as kKPairs / 2
+        // 16-byte chunks of 16 channels each (lane (g, t) reads bytes
+        // [64 m + 16 t, +16): the channel groups kp = 2m, first 8 channels, and
+        // kp = 2m + 1, last 8)
+        constexpr int NL = C::kKPairs / 2;
+        struct Loaded {
+            TileInfo t;
+            int x0;
+            bool ok0, ok8;
+            uint4 a[NL], b[NL];
+            int e0, e8;
+        };
+
+        walk.start(s, e);
+        int jn = 0;
+        // this warp's next tile: every kWarps-th tile of the CTA's range
+        auto next_tile = [&](Loaded& L) -> bool {
+            while (walk.next(L.t)) {
+                if ((jn++ % C::kWarps) == warp) {
+                    L.x0 = walk.x - L.t.count - s;       // slice index of row 0
+                    return true;
+                }
+            }
+            return false;
+        };
+        auto issue = [&](Loaded& L) {
+            const int g = L.t.unit % Hkv;
+            // rows g and g+8 of the tile (clamped inside the tile; extra rows are dropped)
+            const int r0 = gq < L.t.count ? gq : L.t.count - 1;
+            const int r8 = gq + 8 < L.t.count ? gq + 8 : L.t.count - 1;
+            const int p0 = pt[L.x0 + r0], p8 = pt[L.x0 + r8];
+            L.ok0 = p0 >= 0 && p0 < p.s.NPG;
+            L.ok8 = p8 >= 0 && p8 < p.s.NPG;
+            constexpr size_t kRow = 2 * D + 16;
+            const uint8_t* b0 = p.meta8 + ((size_t)(L.ok0 ? p0 : 0) * Hkv + g) * kRow;
+            const uint8_t* b8 = p.meta8 + ((size_t)(L.ok8 ? p8 : 0) * Hkv + g) * kRow;
 #pragma unroll
-        for (int kp = 0; kp < C::kKPairs; ++kp) {
-            xa[kp] = ld_stream_v4(row0 + 64 * kp);
-            xb[kp] = ld_stream_v4(row8 + 64 * kp);
-        }
-        if (t.unit != cur_unit) {
-            cur_unit = t.unit;
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const int head = nb * 8 + gq;
-                const uint32_t* qw = reinterpret_cast<const uint32_t*>(
-                    p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
-#pragma unroll
-                for (int kp = 0; kp < C::kKPairs; ++kp) {
-                    // channels ch0 .. ch0+7 of the [min | max] row; min pairs with q-
-                    const int ch0 = 32 * kp + 8 * tq;
-                    const bool is_max = ch0 >= D;
-                    const int qc = is_max ? ch0 - D : ch0;
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const uint32_t v = head < G ? __ldg(qw + qc / 2 + w) : 0u;
-                        qf[kp][nb][w] = is_max ? pos_part(v) : neg_part(v);
+            for (int m = 0; m < NL; ++m) {
+                L.a[m] = ld_stream_v4(b0 + 64 * m + 16 * tq);
+                L.b[m] = ld_stream_v4(b8 + 64 * m + 16 * tq);
+            }
+            L.e0 = ld_stream_s32(b0 + 2 * D);
+            L.e8 = ld_stream_s32(b8 + 2 * D);
+        };
+        auto process = [&](const Loaded& L) {
+            const TileInfo& t = L.t;
+            const int b = t.unit / Hkv, g = t.unit % Hkv;
+            if (t.unit != cur_unit) {
+                cur_unit = t.unit;
+    #pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    const int head = nb * 8 + gq;
+                    const uint32_t* qw = reinterpret_cast<const uint32_t*>(
+                        p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
+    #pragma unroll
+                    for (int kp = 0; kp < C::kKPairs; ++kp) {
+                        // channels ch0 .. ch0+7 of the [min | max] row; min pairs with q-
+                        const int ch0 = 64 * (kp >> 1) + 16 * tq + 8 * (kp & 1);
+                        const bool is_max = ch0 >= D;
+                        const int qc = is_max ? ch0 - D : ch0;
+    #pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const uint32_t v = head < G ? __ldg(qw + qc / 2 + w) : 0u;
+                            const uint32_t part = is_max ? pos_part(v) : neg_part(v);
+                            qf[kp][nb][w] = bf16x2_to_f16x2(part);
+                        }
                     }
                 }
             }
-        }
-        float acc[NB][4];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-#pragma unroll
-        for (int kp = 0; kp < C::kKPairs; ++kp) {
-            const uint32_t a0[4] = {xa[kp].x, xb[kp].x, xa[kp].y, xb[kp].y};
-            const uint32_t a1[4] = {xa[kp].z, xb[kp].z, xa[kp].w, xb[kp].w};
-#pragma unroll
+            float acc[NB][4];
+    #pragma unroll
+            for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+    #pragma unroll
+            for (int kp = 0; kp < C::kKPairs; ++kp) {
+                const uint4 va = L.a[kp >> 1], vb = L.b[kp >> 1];
+                const uint4 ta = (kp & 1) ? e4m3x8_to_f16x8(va.z, va.w) : e4m3x8_to_f16x8(va.x, va.y);
+                const uint4 tb = (kp & 1) ? e4m3x8_to_f16x8(vb.z, vb.w) : e4m3x8_to_f16x8(vb.x, vb.y);
+                const uint32_t a0[4] = {ta.x, tb.x, ta.y, tb.y};
+                const uint32_t a1[4] = {ta.z, tb.z, ta.w, tb.w};
+    #pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    mma_f16_16816(acc[nb], a0, qf[kp][nb][0], qf[kp][nb][1]);
+                    mma_f16_16816(acc[nb], a1, qf[kp][nb][2], qf[kp][nb][3]);
+                }
+            }
+            const float sc0 = ldexpf(1.f, L.e0), sc8 = ldexpf(1.f, L.e8);
+    #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-                mma_bf16_16816(acc[nb], a0, qf[kp][nb][0], qf[kp][nb][1]);
-                mma_bf16_16816(acc[nb], a1, qf[kp][nb][2], qf[kp][nb][3]);
+                acc[nb][0] *= sc0;
+                acc[nb][1] *= sc0;
+                acc[nb][2] *= sc8;
+                acc[nb][3] *= sc8;
             }
-        }
-        // max over the group's heads: this lane holds heads 8nb + 2tq, +1
-        float m0 = -INFINITY, m8 = -INFINITY;
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-            const int h = nb * 8 + 2 * tq;
-            if (h < G) {
-                m0 = fmaxf(m0, acc[nb][0]);
-                m8 = fmaxf(m8, acc[nb][2]);
+            // max over the group's heads: this lane holds heads 8nb + 2tq, +1
+            float m0 = -INFINITY, m8 = -INFINITY;
+    #pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int h = nb * 8 + 2 * tq;
+                if (h < G) {
+                    m0 = fmaxf(m0, acc[nb][0]);
+                    m8 = fmaxf(m8, acc[nb][2]);
+                }
+                if (h + 1 < G) {
+                    m0 = fmaxf(m0, acc[nb][1]);
+                    m8 = fmaxf(m8, acc[nb][3]);
+                }
             }
-            if (h + 1 < G) {
-                m0 = fmaxf(m0, acc[nb][1]);
-                m8 = fmaxf(m8, acc[nb][3]);
+            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+            m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
+            m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
+            const int row = tq == 0 ? gq : gq + 8;
+            const bool has = tq < 2 && row < t.count;
+            const bool ok = tq == 0 ? L.ok0 : L.ok8;
+            const float v = ok ? (tq == 0 ? m0 : m8) : -INFINITY;
+            if (has) {
+                if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
+                const size_t o = (size_t)t.unit * MP + t.first + row;
+                p.scores_ws[o] = v;
+                if (p.scores_out) p.scores_out[o] = v;
             }
-        }
-        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-        m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
-        m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
-        const int row = tq == 0 ? gq : gq + 8;
-        const bool has = tq < 2 && row < t.count;
-        const bool ok = tq == 0 ? ok0 : ok8;
-        const float v = ok ? (tq == 0 ? m0 : m8) : -INFINITY;
-        if (has) {
-            if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
-            const size_t o = (size_t)t.unit * MP + t.first + row;
-            p.scores_ws[o] = v;
-            if (p.scores_out) p.scores_out[o] = v;
-        }
-        // the unit's key range for the selection (min kept as ~key, so that
-        // both ends merge with atomicMax from a zeroed word), published once
-        // per warp and unit: per-tile atomics on one word serialise in L2
-        const uint32_t key = order_key(v);
-        if (t.unit != kr_unit) {
-            if (lane == 0 && kr_unit >= 0) {
-                atomicMax(&p.keyrange[kr_unit].x, kr_nmin);
-                atomicMax(&p.keyrange[kr_unit].y, kr_max);
+            // the unit's key range for the selection (min kept as ~key, so that
+            // both ends merge with atomicMax from a zeroed word), published once
+            // per warp and unit: per-tile atomics on one word serialise in L2
+            const uint32_t key = order_key(v);
+            if (t.unit != kr_unit) {
+                if (lane == 0 && kr_unit >= 0) {
+                    atomicMax(&p.keyrange[kr_unit].x, kr_nmin);
+                    atomicMax(&p.keyrange[kr_unit].y, kr_max);
+                }
+                kr_unit = t.unit;
+                kr_nmin = kr_max = 0u;
             }
-            kr_unit = t.unit;
-            kr_nmin = kr_max = 0u;
+            kr_nmin = max(kr_nmin, __reduce_max_sync(0xffffffffu, has ? ~key : 0u));
+            kr_max = max(kr_max, __reduce_max_sync(0xffffffffu, has ? key : 0u));
+        };
+        // two tiles in flight per warp: the next tile's loads go out before
+        // the current tile is processed (the fp8 tile needs half the registers)
+        Loaded A, Bt;
+        bool ha = next_tile(A);
+        if (ha) issue(A);
+        while (ha) {
+            const bool hb = next_tile(Bt);
+            if (hb) issue(Bt);
+            process(A);
+            if (!hb) break;
+            ha = next_tile(A);
+            if (ha) issue(A);
+            process(Bt);
         }
-        kr_nmin = max(kr_nmin, __reduce_max_sync(0xffffffffu, has ? ~key : 0u));
-        kr_max = max(kr_max, __reduce_max_sync(0xffffffffu, has ? key : 0u));
+    } else {
+        // bf16: one tile in flight per warp (its registers allow no more)
+        walk.start(s, e);
+        TileInfo t;
+        for (int j = 0; walk.next(t); ++j) {
+            if (j % C::kWarps != warp) continue;
+            const int b = t.unit / Hkv, g = t.unit % Hkv;
+            const int x0 = walk.x - t.count - s;           // slice index of row 0
+            // rows g and g+8 of the tile (clamped inside the tile; extra rows are dropped)
+            const int r0 = gq < t.count ? gq : t.count - 1;
+            const int r8 = gq + 8 < t.count ? gq + 8 : t.count - 1;
+            const int p0 = pt[x0 + r0], p8 = pt[x0 + r8];
+            const bool ok0 = p0 >= 0 && p0 < p.s.NPG, ok8 = p8 >= 0 && p8 < p.s.NPG;
+            const char* row0 = reinterpret_cast<const char*>(
+                p.meta + ((size_t)(ok0 ? p0 : 0) * Hkv + g) * 2 * D) + 16 * tq;
+            const char* row8 = reinterpret_cast<const char*>(
+                p.meta + ((size_t)(ok8 ? p8 : 0) * Hkv + g) * 2 * D) + 16 * tq;
+            uint4 xa[C::kKPairs], xb[C::kKPairs];
+    #pragma unroll
+            for (int kp = 0; kp < C::kKPairs; ++kp) {
+                xa[kp] = ld_stream_v4(row0 + 64 * kp);
+                xb[kp] = ld_stream_v4(row8 + 64 * kp);
+            }
+            if (t.unit != cur_unit) {
+                cur_unit = t.unit;
+    #pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    const int head = nb * 8 + gq;
+                    const uint32_t* qw = reinterpret_cast<const uint32_t*>(
+                        p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
+    #pragma unroll
+                    for (int kp = 0; kp < C::kKPairs; ++kp) {
+                        // channels ch0 .. ch0+7 of the [min | max] row; min pairs with q-
+                        const int ch0 = 32 * kp + 8 * tq;
+                        const bool is_max = ch0 >= D;
+                        const int qc = is_max ? ch0 - D : ch0;
+    #pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const uint32_t v = head < G ? __ldg(qw + qc / 2 + w) : 0u;
+                            qf[kp][nb][w] = is_max ? pos_part(v) : neg_part(v);
+                        }
+                    }
+                }
+            }
+            float acc[NB][4];
+    #pragma unroll
+            for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+    #pragma unroll
+            for (int kp = 0; kp < C::kKPairs; ++kp) {
+                const uint32_t a0[4] = {xa[kp].x, xb[kp].x, xa[kp].y, xb[kp].y};
+                const uint32_t a1[4] = {xa[kp].z, xb[kp].z, xa[kp].w, xb[kp].w};
+    #pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    mma_bf16_16816(acc[nb], a0, qf[kp][nb][0], qf[kp][nb][1]);
+                    mma_bf16_16816(acc[nb], a1, qf[kp][nb][2], qf[kp][nb][3]);
+                }
+            }
+            // max over the group's heads: this lane holds heads 8nb + 2tq, +1
+            float m0 = -INFINITY, m8 = -INFINITY;
+    #pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int h = nb * 8 + 2 * tq;
+                if (h < G) {
+                    m0 = fmaxf(m0, acc[nb][0]);
+                    m8 = fmaxf(m8, acc[nb][2]);
+                }
+                if (h + 1 < G) {
+                    m0 = fmaxf(m0, acc[nb][1]);
+                    m8 = fmaxf(m8, acc[nb][3]);
+                }
+            }
+            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+            m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
+            m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
+            const int row = tq == 0 ? gq : gq + 8;
+            const bool has = tq < 2 && row < t.count;
+            const bool ok = tq == 0 ? ok0 : ok8;
+            const float v = ok ? (tq == 0 ? m0 : m8) : -INFINITY;
+            if (has) {
+                if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
+                const size_t o = (size_t)t.unit * MP + t.first + row;
+                p.scores_ws[o] = v;
+                if (p.scores_out) p.scores_out[o] = v;
+            }
+            // the unit's key range for the selection (min kept as ~key, so that
+            // both ends merge with atomicMax from a zeroed word), published once
+            // per warp and unit: per-tile atomics on one word serialise in L2
+            const uint32_t key = order_key(v);
+            if (t.unit != kr_unit) {
+                if (lane == 0 && kr_unit >= 0) {
+                    atomicMax(&p.keyrange[kr_unit].x, kr_nmin);
+                    atomicMax(&p.keyrange[kr_unit].y, kr_max);
+                }
+                kr_unit = t.unit;
+                kr_nmin = kr_max = 0u;
+            }
+            kr_nmin = max(kr_nmin, __reduce_max_sync(0xffffffffu, has ? ~key : 0u));
+            kr_max = max(kr_max, __reduce_max_sync(0xffffffffu, has ? key : 0u));
+        }
     }
     if (lane == 0 && kr_unit >= 0) {
         atomicMax(&p.keyrange[kr_unit].x, kr_nmin);
@@ -303,10 +491,10 @@ score_kernel(ScoreParams p) {
     }
 }
 
-template <int D, int NB>
+template <int D, int NB, bool F8>
 cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t st) {
     using C = ScoreCfg<D, NB>;
-    auto kern = score_kernel<D, NB>;
+    auto kern = score_kernel<D, NB, F8>;
     static int attr_done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -330,12 +518,18 @@ cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t st) {
 cudaError_t launch_score(const ScoreParams& p, cudaStream_t st) {
     const int nb = p.s.G > 8 ? 2 : 1;
     switch (p.s.D * 10 + nb) {
-        case 641: return launch_score_t<64, 1>(p, st);
-        case 642: return launch_score_t<64, 2>(p, st);
-        case 1281: return launch_score_t<128, 1>(p, st);
-        case 1282: return launch_score_t<128, 2>(p, st);
-        case 2561: return launch_score_t<256, 1>(p, st);
-        case 2562: return launch_score_t<256, 2>(p, st);
+        case 641: return p.meta8 ? launch_score_t<64, 1, true>(p, st)
+                          : launch_score_t<64, 1, false>(p, st);
+        case 642: return p.meta8 ? launch_score_t<64, 2, true>(p, st)
+                          : launch_score_t<64, 2, false>(p, st);
+        case 1281: return p.meta8 ? launch_score_t<128, 1, true>(p, st)
+                          : launch_score_t<128, 1, false>(p, st);
+        case 1282: return p.meta8 ? launch_score_t<128, 2, true>(p, st)
+                          : launch_score_t<128, 2, false>(p, st);
+        case 2561: return p.meta8 ? launch_score_t<256, 1, true>(p, st)
+                          : launch_score_t<256, 1, false>(p, st);
+        case 2562: return p.meta8 ? launch_score_t<256, 2, true>(p, st)
+                          : launch_score_t<256, 2, false>(p, st);
         default: return cudaErrorInvalidValue;
     }
 }

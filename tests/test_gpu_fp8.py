@@ -1,0 +1,145 @@
+"""GPU parity of the optional fp8 metadata path against the oracle's fp8
+definition (csa_oracle.c): the fp8 copy bit-exact (after a rebuild and after
+appends), scores to fp32 accuracy, the selection by the band rule, and the
+one-call output in every unit whose selection is the oracle's own."""
+import math
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_decoding_b200 import csa
+from long_context_decoding_b200 import workloads as wl
+from parity import PS, assert_out_close, assert_scores_close, check_selection
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    oracle.set_threads(0)
+    yield
+
+
+class Fp8Run:
+    def __init__(self, case: wl.Case, budget=None):
+        self.c = c = case
+        w = case.w
+        self.budget = case.budget if budget is None else budget
+        self.max_sel = max(1, max(w.max_sel, self.budget // PS))
+        self.d = csa.make_dims(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.num_pages, self.max_sel)
+        self.od = oracle.Dims(w.B, w.Hq, w.Hkv, w.D, PS, w.max_pages, w.num_pages)
+        self.layer = csa.Layer(self.d, c.k_cache, c.v_cache, c.page_table, c.seq_lens, w.prefix,
+                               case.window, self.budget, fp8=True)
+        self.layer.rebuild_meta()
+
+    def host(self):
+        c = self.c
+        return dict(q=wl.bits(c.q), k=wl.bits(c.k_cache), v=wl.bits(c.v_cache),
+                    pt=c.page_table.cpu().numpy(), sl=c.seq_lens.cpu().numpy())
+
+    def oracle_meta8(self, h):
+        m = oracle.meta(self.od, h["k"], h["pt"], h["sl"])
+        return oracle.meta_fp8(self.od, m, h["pt"], h["sl"])
+
+
+def assert_meta8_equal(run: Fp8Run, h):
+    ref = run.oracle_meta8(h)
+    got = run.layer.meta8.cpu().numpy()
+    for b in range(run.d.B):
+        np_b = -(-int(h["sl"][b]) // PS)
+        phys = h["pt"][b, :np_b]
+        np.testing.assert_array_equal(got[phys], ref[phys], err_msg=f"fp8 metadata, sequence {b}")
+
+
+def check_fp8(run: Fp8Run, one_call=True):
+    h = run.host()
+    assert_meta8_equal(run, h)
+    w = run.c.w
+    ref = oracle.step_fp8(run.od, h["q"], h["k"], h["v"], h["pt"], h["sl"], w.prefix,
+                          run.c.window, run.budget, run.max_sel, 1.0 / math.sqrt(w.D))
+    sc = torch.full((run.d.B, run.d.Hkv, run.d.max_pages_per_seq), float("nan"),
+                    dtype=torch.float32, device=run.c.q.device)
+    lay = run.layer
+    csa.score_select_fp8(run.d, run.c.q, lay.meta8, run.c.page_table, run.c.seq_lens, w.prefix,
+                         run.c.window, run.budget, lay.sel, lay.n_sel, lay.ws, scores_out=sc)
+    torch.cuda.synchronize()
+    assert_scores_close(sc, ref["scores"])
+    check_selection(lay.sel, lay.n_sel, ref["scores"], ref["sel"], ref["nsel"], gpu_scores=sc)
+    sel_s, nsel_s = lay.sel.clone(), lay.n_sel.clone()
+    if not one_call:
+        return 0
+    out = lay.step(run.c.q, fused=True)
+    torch.cuda.synchronize()
+    assert csa.device_status(lay.ws) == 0
+    assert torch.equal(lay.n_sel, nsel_s)
+    gs, gn = lay.sel.cpu().numpy(), lay.n_sel.cpu().numpy()
+    assert all(np.array_equal(gs[b, g, :gn[b, g]], sel_s.cpu().numpy()[b, g, :gn[b, g]])
+               for b in range(run.d.B) for g in range(run.d.Hkv))
+    G = w.Hq // w.Hkv
+    same = 0
+    for b in range(run.d.B):
+        for g in range(run.d.Hkv):
+            k = int(gn[b, g])
+            if not np.array_equal(gs[b, g, :k], ref["sel"][b, g, :k]):
+                continue
+            same += 1
+            hh = slice(g * G, (g + 1) * G)
+            assert_out_close(out[b, hh], lay.lse[b, hh], ref["out"][b, hh], ref["lse"][b, hh],
+                             f"fp8 one-call, unit ({b},{g})")
+    return same
+
+
+@pytest.mark.parametrize("w", [wl.TINY, wl.CTX32K, wl.CTX64K], ids=lambda w: w.name)
+def test_fp8_parity(w, cuda):
+    same = check_fp8(Fp8Run(wl.make_case(w, cuda)))
+    if w is not wl.TINY:
+        assert same >= 1
+
+
+@pytest.mark.parametrize("G", [1, 8, 16])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_fp8_group_sizes_and_head_dims(G, D, cuda):
+    w = wl.Workload("fp8", B=2, Hq=2 * G, Hkv=2, D=D, seq_lens=(3000, 2049), prefix=40,
+                    window=100, budget=480, seed=13)
+    check_fp8(Fp8Run(wl.make_case(w, cuda)))
+
+
+def test_fp8_copy_after_appends_matches_rebuild(cuda):
+    """64 single-token appends through csa_meta_update_fp8: the fp8 copy is
+    the oracle's from the final cache, bit for bit."""
+    w = replace(wl.CTX32K, steps=64)
+    case = wl.make_case(w, cuda)
+    run = Fp8Run(case)
+    d, lay = run.d, run.layer
+    for s in range(64):
+        _, nk, nv = wl.step_tokens(case, s)
+        case.seq_lens += 1
+        csa.meta_update_fp8(d, case.k_cache, case.v_cache, lay.meta, lay.meta8, case.page_table,
+                            case.seq_lens, nk, nv, 1, lay.ws)
+    torch.cuda.synchronize()
+    assert csa.device_status(lay.ws) == 0
+    assert_meta8_equal(run, run.host())
+
+
+def test_fp8_scores_bound_the_bf16_scores(cuda):
+    """On the GPU, too: the fp8 score of every candidate is at least its bf16
+    score (the box only grows)."""
+    case = wl.make_case(wl.CTX32K, cuda)
+    run = Fp8Run(case)
+    d, lay, w = run.d, run.layer, case.w
+    s8 = torch.full((d.B, d.Hkv, d.max_pages_per_seq), float("nan"), device=cuda)
+    s16 = torch.full_like(s8, float("nan"))
+    csa.score_select_fp8(d, case.q, lay.meta8, case.page_table, case.seq_lens, w.prefix,
+                         case.window, run.budget, lay.sel, lay.n_sel, lay.ws, scores_out=s8)
+    csa.score_select(d, case.q, lay.meta, case.page_table, case.seq_lens, w.prefix, case.window,
+                     run.budget, lay.sel, lay.n_sel, lay.ws, scores_out=s16)
+    torch.cuda.synchronize()
+    cand = ~torch.isnan(s16)
+    assert torch.equal(cand, ~torch.isnan(s8))
+    # fp32 sums of exact products: allow their rounding
+    assert (s8[cand] >= s16[cand] - 1e-5 * s16[cand].abs() - 1e-3).all()
