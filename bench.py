@@ -447,7 +447,7 @@ def run_ours(args, dist: Dist, base: wl.Workload):
                             "gbs": dec_bytes / times["decode"] / 1e9}}
         ach = calls["score"]["gbs"]
         traffic, traffic_src = score_traffic()
-        line["roofline"] = {"bound": "hbm", "kernel": "score_kernel (Quest scoring)",
+        line["roofline"] = {"bound": "hbm", "kernel": "score_direct_kernel (Quest scoring)",
                             "achieved": ach, "peak": peak, "peak_kind": peak_kind,
                             "unit": "GB/s", "frac": ach / peak, "traffic": traffic,
                             "traffic_source": (f"ncu dram__bytes_read+write per launch, {traffic_src}, "

@@ -94,20 +94,6 @@ __host__ __device__ __forceinline__ size_t record_stride(int G, int D) {
     return ((size_t)G * D + 2 * G + 3) & ~(size_t)3;
 }
 
-// ------------------------------------------------------------ page copies
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // Issues the cp.async copies of one page's K and V tiles (16 tokens x D) into
 // a swizzled buffer; token rows >= rows_valid are zero-filled.
 template <int D>

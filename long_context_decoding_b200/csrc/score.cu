@@ -13,37 +13,31 @@
 // are exact in fp32; fp32 accumulation), and the kv-head score is the max
 // over the group's heads.
 //
-// Data path.  The kernel streams 4*D bytes of metadata per candidate page
-// from random physical pages and does ~2 flop per byte: it is HBM-bound, and
-// what decides its speed is how many bytes are in flight.  Every warp of the
-// grid loads its own tiles straight into the registers that feed the MMA:
-// with the k index of the contraction permuted (the same permutation on the
-// q side), lane (g, t) of a warp needs exactly the 16-byte chunks
-// t, t+4, t+8, ... of rows g and g+8 of the tile, so a tile is 2D/16 plain
-// 16-byte loads per lane (non-allocating in L1), with no shared-memory
-// staging and no barriers.  Measured on B200 for 16 x 512-byte rows this
-// sustains ~81% of the copy peak, where a TMA bulk copy per row (512 bytes)
-// is limited by its per-copy issue cost to ~30%.
-//   * the candidates of all (sequence, kv-head) units are flattened and split
-//     evenly over a grid that fills every SM;
-//   * each CTA copies its slice of the page table into shared memory once;
-//   * warps take the CTA's 16-page tiles round-robin.
+// Data path.  The kernels stream one metadata row per candidate (page,
+// kv-head) from random physical pages and do ~2 flop per byte: they are
+// bound by memory, and on B200 the rate of random row requests (~12 G rows/s
+// for rows of 256 to 512 bytes) matters as much as the bytes.  Two load
+// paths, chosen per shape by measurement:
+//   * direct (bf16 metadata, D <= 128): every warp loads its own tiles
+//     straight into the registers that feed the MMA.  With the k index of the
+//     contraction permuted (the same permutation on the q side), lane (g, t)
+//     needs exactly the 16-byte chunks t, t+4, ... of rows g and g+8, so a
+//     tile is 2D/16 plain 16-byte loads per lane, with no staging and no
+//     barriers.
+//   * ring (bf16 metadata at D = 256, and the fp8 copy): each warp copies
+//     whole rows of its tiles into a private shared-memory ring with 16-byte
+//     cp.async (one 512-byte row per instruction), keeps several tiles in
+//     flight, and reads a landed tile into MMA fragments with ldmatrix.
+// Both: the candidates of all (sequence, kv-head) units are flattened and
+// split evenly over the grid; each CTA copies its slice of the page table
+// into shared memory once, before the dependency wait.  A TMA bulk copy per
+// row (512 bytes) is limited by its per-copy issue cost to ~30% of the copy
+// peak on B200, so neither path uses one.
 #include "common.cuh"
 #include "internal.h"
 
 namespace csa {
 namespace {
-
-template <int D, int NB>
-struct ScoreCfg {
-    static constexpr int kWarps = 8;
-    static constexpr int kThreads = 32 * kWarps;
-    static constexpr int kKPairs = 2 * D / 32;        // 32-channel steps along [min | max]
-    // page-table slice | 3 x [B + 1] ints
-    static __host__ __device__ size_t smem_bytes(int B) {
-        return (size_t)kScorePtCap * 4 + 3 * 4 * (size_t)(B + 1);
-    }
-};
 
 struct TileInfo {
     int unit;      // b * Hkv + g
@@ -64,9 +58,33 @@ __device__ __forceinline__ uint32_t pos_part(uint32_t w) {   // max(q, 0) per bf
     return r;
 }
 
-// Walks the CTA's range [x, e) of the flattened candidate list in tiles that
-// never cross a (sequence, kv-head) unit.  One division at start-up; every
-// step after that is a few integer adds.
+// Two E4M3 values (bytes 0 and 1 of w) -> f16x2, exactly (hardware cvt).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h2)
+        : "r"(w));
+    return h2;
+}
+// bf16x2 -> f16x2 (exact for |x| in [2^-17, 65504]; larger values saturate).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(bf16_hi(w)), "f"(bf16_lo(w)));
+    return r;
+}
+
+// 16-byte load that does not allocate in L1 (the metadata is read once).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Walks a range [x, e) of the flattened candidate list in tiles that never
+// cross a (sequence, kv-head) unit.  One division at start-up; every step
+// after that is a few integer adds.
 struct TileWalker {
     int x, e;
     const int* seq_off;   // [B + 1]: first flattened index of sequence b
@@ -115,64 +133,25 @@ struct TileWalker {
     }
 };
 
-// 16-byte load that does not allocate in L1 (the metadata is read once).
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
+// Shared memory common to both kernels: page-table slice | 3 x [B + 1] ints.
+__host__ __device__ __forceinline__ size_t score_common_bytes(int B) {
+    return (size_t)kScorePtCap * 4 + 12 * (size_t)(B + 1);
 }
 
-// 4-byte load that does not allocate in L1 (the fp8 row exponent).
-__device__ __forceinline__ int ld_stream_s32(const void* p) {
-    int v;
-    asm volatile("ld.global.nc.L1::no_allocate.s32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
-
-// Two E4M3 values (bytes 0 and 1 of w) -> f16x2, exactly (hardware cvt).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
-    uint32_t h2;
-    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
-        : "=r"(h2)
-        : "r"(w));
-    return h2;
-}
-// 8 E4M3 channels -> 8 f16 channels in the order of a 16-byte chunk.
-__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint32_t lo, uint32_t hi) {
-    return make_uint4(e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi),
-                      e4m3x2_to_f16x2(hi >> 16));
-}
-// bf16x2 -> f16x2 (exact for |x| in [2^-17, 65504]; larger values saturate).
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
-    uint32_t r;
-    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(bf16_hi(w)), "f"(bf16_lo(w)));
-    return r;
-}
-
-// F8: the metadata is the fp8 copy (rows of 2D E4M3 bytes + a 16-byte trailer
-// whose first int32 is the row's exponent e): 16 channels per 16-byte load,
-// converted by the hardware to f16 (one instruction per two channels; the
-// three-step route to bf16 made the conversions the bottleneck), multiplied
-// with q in f16 on the tensor cores (products exact in fp32; q is exact in
-// f16 for |q| >= 2^-17), and the row's sums scaled by 2^e.
-template <int D, int NB, bool F8>
-__global__ void __launch_bounds__(ScoreCfg<D, NB>::kThreads,
-                                  ((NB == 1 && !(F8 && D == 256)) || D == 64) ? 2 : 1)
-score_kernel(ScoreParams p) {
-    using C = ScoreCfg<D, NB>;
-    extern __shared__ __align__(16) int smem_i[];
+// The prologue of both kernels: candidates per sequence, their exclusive scan
+// over (sequence, kv-head), this CTA's range [s, e) of the flattened list and
+// its page-table slice -- all from caller inputs, before the dependency wait
+// -- then the wait (the metadata was written by the previous kernel on the
+// stream).  Returns the walker template (range not started).
+__device__ __forceinline__ TileWalker score_setup(const ScoreParams& p, int* smem_i, int& s,
+                                                  int& e) {
+    const int B = p.s.B, Hkv = p.s.Hkv, MP = p.s.MP;
+    const int tid = threadIdx.x, lane = tid & 31, nthr = blockDim.x;
     int* pt = smem_i;
     int* seq_n = pt + kScorePtCap;
-    int* seq_clo = seq_n + (p.s.B + 1);
-    int* seq_off = seq_clo + (p.s.B + 1);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int B = p.s.B, Hkv = p.s.Hkv, G = p.s.G, MP = p.s.MP;
-
-    // Candidates per sequence (caller inputs only before the dependency wait).
-    for (int b = tid; b < B; b += C::kThreads) {
+    int* seq_clo = seq_n + (B + 1);
+    int* seq_off = seq_clo + (B + 1);
+    for (int b = tid; b < B; b += nthr) {
         int L = p.seq_lens[b];
         if (L < 0 || L > MP * kPage) {
             latch_flag(p.flags, CSA_DEVFLAG_BAD_SEQ_LEN);
@@ -183,7 +162,7 @@ score_kernel(ScoreParams p) {
         seq_clo[b] = sg.c_lo;
     }
     __syncthreads();
-    if (warp == 0) {   // exclusive scan of Hkv * n_b
+    if (tid < 32) {   // exclusive scan of Hkv * n_b
         int carry = 0;
         for (int base = 0; base < B; base += 32) {
             const int b = base + lane;
@@ -201,7 +180,8 @@ score_kernel(ScoreParams p) {
     }
     __syncthreads();
     const long long N = seq_off[B];
-    const int s = (int)(N * blockIdx.x / gridDim.x), e = (int)(N * (blockIdx.x + 1) / gridDim.x);
+    s = (int)(N * blockIdx.x / gridDim.x);
+    e = (int)(N * (blockIdx.x + 1) / gridDim.x);
 
     TileWalker walk;
     walk.seq_off = seq_off;
@@ -218,299 +198,430 @@ score_kernel(ScoreParams p) {
         int at = 0;
         while (fill.next(run, 1 << 30)) {
             const int32_t* src = p.page_table + (size_t)(run.unit / Hkv) * MP + run.first;
-            for (int i = tid; i < run.count; i += C::kThreads) pt[at + i] = __ldg(src + i);
+            for (int i = tid; i < run.count; i += nthr) pt[at + i] = __ldg(src + i);
             at += run.count;
         }
     }
-    // the metadata was written by the previous kernel on the stream
     pdl_wait();
     pdl_launch_dependents();
     __syncthreads();
-    if (s >= e) return;
+    return walk;
+}
 
+// The unit's key range for the selection, merged per warp: the minimum kept
+// as ~key, so that both ends merge with atomicMax from a zeroed word, and
+// published once per warp and unit (per-tile atomics on one word serialise
+// in L2).
+struct KeyRange {
+    int unit = -1;
+    uint32_t nmin = 0u, max = 0u;
+    __device__ void flush(const ScoreParams& p, int lane) {
+        if (lane == 0 && unit >= 0) {
+            atomicMax(&p.keyrange[unit].x, nmin);
+            atomicMax(&p.keyrange[unit].y, max);
+        }
+    }
+};
+
+// Tile epilogue of both kernels.  acc holds the MMA results (rows g, g+8 x
+// heads 8 nb + 2t, +1); the kv-head score of a row is the max over the
+// group's heads.  Rows with a bad page id score -inf and raise the flag.
+template <int NB>
+__device__ __forceinline__ void score_store(const ScoreParams& p, const TileInfo& t,
+                                            const float (&acc)[NB][4], bool ok0, bool ok8,
+                                            KeyRange& kr, int lane) {
+    const int gq = lane >> 2, tq = lane & 3, G = p.s.G;
+    float m0 = -INFINITY, m8 = -INFINITY;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        const int h = nb * 8 + 2 * tq;
+        if (h < G) {
+            m0 = fmaxf(m0, acc[nb][0]);
+            m8 = fmaxf(m8, acc[nb][2]);
+        }
+        if (h + 1 < G) {
+            m0 = fmaxf(m0, acc[nb][1]);
+            m8 = fmaxf(m8, acc[nb][3]);
+        }
+    }
+    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+    m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
+    m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
+    const int row = tq == 0 ? gq : gq + 8;
+    const bool has = tq < 2 && row < t.count;
+    const bool ok = tq == 0 ? ok0 : ok8;
+    const float v = ok ? (tq == 0 ? m0 : m8) : -INFINITY;
+    if (has) {
+        if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
+        const size_t o = (size_t)t.unit * p.s.MP + t.first + row;
+        p.scores_ws[o] = v;
+        if (p.scores_out) p.scores_out[o] = v;
+    }
+    const uint32_t key = order_key(v);
+    if (t.unit != kr.unit) {
+        kr.flush(p, lane);
+        kr.unit = t.unit;
+        kr.nmin = kr.max = 0u;
+    }
+    kr.nmin = max(kr.nmin, __reduce_max_sync(0xffffffffu, has ? ~key : 0u));
+    kr.max = max(kr.max, __reduce_max_sync(0xffffffffu, has ? key : 0u));
+}
+
+// Whether row r of a tile starting at slice index x0 has a valid page id (ph:
+// the id of row min(r, count - 1)).
+__device__ __forceinline__ bool row_ok(const ScoreParams& p, const int* pt, int x0, int r,
+                                       int count, int& ph) {
+    ph = pt[x0 + (r < count ? r : count - 1)];
+    return ph >= 0 && ph < p.s.NPG;
+}
+
+// ------------------------------------------------------------ direct path
+// bf16 metadata; 8 warps per CTA, tiles round-robin over the CTA's warps.
+template <int D, int NB>
+struct DirectCfg {
+    static constexpr int kWarps = 8;
+    static constexpr int kThreads = 32 * kWarps;
+    static constexpr int kKPairs = 2 * D / 32;        // 32-channel steps along [min | max]
+    static constexpr int kMinBlocks = (NB == 1 || D == 64) ? 2 : 1;
+    static __host__ __device__ size_t smem_bytes(int B) { return score_common_bytes(B); }
+};
+
+template <int D, int NB>
+__global__ void __launch_bounds__(DirectCfg<D, NB>::kThreads, DirectCfg<D, NB>::kMinBlocks)
+score_direct_kernel(ScoreParams p) {
+    using C = DirectCfg<D, NB>;
+    extern __shared__ __align__(16) int smem_i[];
+    int s, e;
+    TileWalker walk = score_setup(p, smem_i, s, e);
+    if (s >= e) return;
+    const int* pt = smem_i;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int Hkv = p.s.Hkv, G = p.s.G;
     const int gq = lane >> 2, tq = lane & 3;
     uint32_t qf[C::kKPairs][NB][4];          // B fragments of [q- | q+] for the current unit
     int cur_unit = -1;
-    int kr_unit = -1;                        // key range of this warp's current unit
-    uint32_t kr_nmin = 0u, kr_max = 0u;
-    if constexpr (F8) {
-        // registers of one tile: rows g and g+8 of the fp8 copy as kKPairs / 2
-        // 16-byte chunks of 16 channels each (lane (g, t) reads bytes
-        // [64 m + 16 t, +16): the channel groups kp = 2m, first 8 channels, and
-        // kp = 2m + 1, last 8)
-        constexpr int NL = C::kKPairs / 2;
-        struct Loaded {
-            TileInfo t;
-            int x0;
-            bool ok0, ok8;
-            uint4 a[NL], b[NL];
-            int e0, e8;
-        };
+    KeyRange kr;
 
-        walk.start(s, e);
-        int jn = 0;
-        // this warp's next tile: every kWarps-th tile of the CTA's range
-        auto next_tile = [&](Loaded& L) -> bool {
-            while (walk.next(L.t)) {
-                if ((jn++ % C::kWarps) == warp) {
-                    L.x0 = walk.x - L.t.count - s;       // slice index of row 0
-                    return true;
-                }
-            }
-            return false;
-        };
-        auto issue = [&](Loaded& L) {
-            const int g = L.t.unit % Hkv;
-            // rows g and g+8 of the tile (clamped inside the tile; extra rows are dropped)
-            const int r0 = gq < L.t.count ? gq : L.t.count - 1;
-            const int r8 = gq + 8 < L.t.count ? gq + 8 : L.t.count - 1;
-            const int p0 = pt[L.x0 + r0], p8 = pt[L.x0 + r8];
-            L.ok0 = p0 >= 0 && p0 < p.s.NPG;
-            L.ok8 = p8 >= 0 && p8 < p.s.NPG;
-            constexpr size_t kRow = 2 * D + 16;
-            const uint8_t* b0 = p.meta8 + ((size_t)(L.ok0 ? p0 : 0) * Hkv + g) * kRow;
-            const uint8_t* b8 = p.meta8 + ((size_t)(L.ok8 ? p8 : 0) * Hkv + g) * kRow;
+    walk.start(s, e);
+    TileInfo t;
+    for (int j = 0; walk.next(t); ++j) {
+        if (j % C::kWarps != warp) continue;
+        const int b = t.unit / Hkv, g = t.unit % Hkv;
+        const int x0 = walk.x - t.count - s;           // slice index of row 0
+        // rows g and g+8 of the tile (clamped inside the tile; extra rows are dropped)
+        int p0, p8;
+        const bool ok0 = row_ok(p, pt, x0, gq, t.count, p0);
+        const bool ok8 = row_ok(p, pt, x0, gq + 8, t.count, p8);
+        const char* row0 = reinterpret_cast<const char*>(
+            p.meta + ((size_t)(ok0 ? p0 : 0) * Hkv + g) * 2 * D) + 16 * tq;
+        const char* row8 = reinterpret_cast<const char*>(
+            p.meta + ((size_t)(ok8 ? p8 : 0) * Hkv + g) * 2 * D) + 16 * tq;
+        uint4 xa[C::kKPairs], xb[C::kKPairs];
 #pragma unroll
-            for (int m = 0; m < NL; ++m) {
-                L.a[m] = ld_stream_v4(b0 + 64 * m + 16 * tq);
-                L.b[m] = ld_stream_v4(b8 + 64 * m + 16 * tq);
-            }
-            L.e0 = ld_stream_s32(b0 + 2 * D);
-            L.e8 = ld_stream_s32(b8 + 2 * D);
-        };
-        auto process = [&](const Loaded& L) {
-            const TileInfo& t = L.t;
-            const int b = t.unit / Hkv, g = t.unit % Hkv;
-            if (t.unit != cur_unit) {
-                cur_unit = t.unit;
-    #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    const int head = nb * 8 + gq;
-                    const uint32_t* qw = reinterpret_cast<const uint32_t*>(
-                        p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
-    #pragma unroll
-                    for (int kp = 0; kp < C::kKPairs; ++kp) {
-                        // channels ch0 .. ch0+7 of the [min | max] row; min pairs with q-
-                        const int ch0 = 64 * (kp >> 1) + 16 * tq + 8 * (kp & 1);
-                        const bool is_max = ch0 >= D;
-                        const int qc = is_max ? ch0 - D : ch0;
-    #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const uint32_t v = head < G ? __ldg(qw + qc / 2 + w) : 0u;
-                            const uint32_t part = is_max ? pos_part(v) : neg_part(v);
-                            qf[kp][nb][w] = bf16x2_to_f16x2(part);
-                        }
+        for (int kp = 0; kp < C::kKPairs; ++kp) {
+            xa[kp] = ld_stream_v4(row0 + 64 * kp);
+            xb[kp] = ld_stream_v4(row8 + 64 * kp);
+        }
+        if (t.unit != cur_unit) {
+            cur_unit = t.unit;
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int head = nb * 8 + gq;
+                const uint32_t* qw = reinterpret_cast<const uint32_t*>(
+                    p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
+#pragma unroll
+                for (int kp = 0; kp < C::kKPairs; ++kp) {
+                    // channels ch0 .. ch0+7 of the [min | max] row; min pairs with q-
+                    const int ch0 = 32 * kp + 8 * tq;
+                    const bool is_max = ch0 >= D;
+                    const int qc = is_max ? ch0 - D : ch0;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const uint32_t v = head < G ? __ldg(qw + qc / 2 + w) : 0u;
+                        qf[kp][nb][w] = is_max ? pos_part(v) : neg_part(v);
                     }
                 }
             }
-            float acc[NB][4];
-    #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-    #pragma unroll
-            for (int kp = 0; kp < C::kKPairs; ++kp) {
-                const uint4 va = L.a[kp >> 1], vb = L.b[kp >> 1];
-                const uint4 ta = (kp & 1) ? e4m3x8_to_f16x8(va.z, va.w) : e4m3x8_to_f16x8(va.x, va.y);
-                const uint4 tb = (kp & 1) ? e4m3x8_to_f16x8(vb.z, vb.w) : e4m3x8_to_f16x8(vb.x, vb.y);
-                const uint32_t a0[4] = {ta.x, tb.x, ta.y, tb.y};
-                const uint32_t a1[4] = {ta.z, tb.z, ta.w, tb.w};
-    #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    mma_f16_16816(acc[nb], a0, qf[kp][nb][0], qf[kp][nb][1]);
-                    mma_f16_16816(acc[nb], a1, qf[kp][nb][2], qf[kp][nb][3]);
-                }
-            }
-            const float sc0 = ldexpf(1.f, L.e0), sc8 = ldexpf(1.f, L.e8);
-    #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                acc[nb][0] *= sc0;
-                acc[nb][1] *= sc0;
-                acc[nb][2] *= sc8;
-                acc[nb][3] *= sc8;
-            }
-            // max over the group's heads: this lane holds heads 8nb + 2tq, +1
-            float m0 = -INFINITY, m8 = -INFINITY;
-    #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const int h = nb * 8 + 2 * tq;
-                if (h < G) {
-                    m0 = fmaxf(m0, acc[nb][0]);
-                    m8 = fmaxf(m8, acc[nb][2]);
-                }
-                if (h + 1 < G) {
-                    m0 = fmaxf(m0, acc[nb][1]);
-                    m8 = fmaxf(m8, acc[nb][3]);
-                }
-            }
-            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-            m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
-            m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
-            const int row = tq == 0 ? gq : gq + 8;
-            const bool has = tq < 2 && row < t.count;
-            const bool ok = tq == 0 ? L.ok0 : L.ok8;
-            const float v = ok ? (tq == 0 ? m0 : m8) : -INFINITY;
-            if (has) {
-                if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
-                const size_t o = (size_t)t.unit * MP + t.first + row;
-                p.scores_ws[o] = v;
-                if (p.scores_out) p.scores_out[o] = v;
-            }
-            // the unit's key range for the selection (min kept as ~key, so that
-            // both ends merge with atomicMax from a zeroed word), published once
-            // per warp and unit: per-tile atomics on one word serialise in L2
-            const uint32_t key = order_key(v);
-            if (t.unit != kr_unit) {
-                if (lane == 0 && kr_unit >= 0) {
-                    atomicMax(&p.keyrange[kr_unit].x, kr_nmin);
-                    atomicMax(&p.keyrange[kr_unit].y, kr_max);
-                }
-                kr_unit = t.unit;
-                kr_nmin = kr_max = 0u;
-            }
-            kr_nmin = max(kr_nmin, __reduce_max_sync(0xffffffffu, has ? ~key : 0u));
-            kr_max = max(kr_max, __reduce_max_sync(0xffffffffu, has ? key : 0u));
-        };
-        // two tiles in flight per warp: the next tile's loads go out before
-        // the current tile is processed (the fp8 tile needs half the registers)
-        Loaded A, Bt;
-        bool ha = next_tile(A);
-        if (ha) issue(A);
-        while (ha) {
-            const bool hb = next_tile(Bt);
-            if (hb) issue(Bt);
-            process(A);
-            if (!hb) break;
-            ha = next_tile(A);
-            if (ha) issue(A);
-            process(Bt);
         }
-    } else {
-        // bf16: one tile in flight per warp (its registers allow no more)
-        walk.start(s, e);
+        float acc[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+#pragma unroll
+        for (int kp = 0; kp < C::kKPairs; ++kp) {
+            const uint32_t a0[4] = {xa[kp].x, xb[kp].x, xa[kp].y, xb[kp].y};
+            const uint32_t a1[4] = {xa[kp].z, xb[kp].z, xa[kp].w, xb[kp].w};
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                mma_bf16_16816(acc[nb], a0, qf[kp][nb][0], qf[kp][nb][1]);
+                mma_bf16_16816(acc[nb], a1, qf[kp][nb][2], qf[kp][nb][3]);
+            }
+        }
+        score_store<NB>(p, t, acc, ok0, ok8, kr, lane);
+    }
+    kr.flush(p, lane);
+}
+
+// ------------------------------------------------------------ ring path
+// Shared-memory rings, one per warp, of kStages tiles of 16 rows; each warp
+// takes a contiguous 1/kWarps of the CTA's range.
+template <int D, bool F8>
+struct RingCfg {
+    static constexpr int kRowBytes = F8 ? 2 * D + 16 : 4 * D;   // one (page, kv-head) row
+    static constexpr int kRowChunks = kRowBytes / 16;
+    // shared-memory row stride: an odd number of 16-byte chunks, so that the 8
+    // row addresses of an ldmatrix phase fall in distinct banks
+    static constexpr int kStride = F8 ? kRowBytes : kRowBytes + 16;
+    static constexpr int kTileSmem = 16 * kStride;
+    static constexpr int kTileChunks = 16 * kRowChunks;
+    static constexpr int kCopyIters = (kTileChunks + 31) / 32;
+    static constexpr int kWarps = kTileSmem > 12 * 1024 ? 2 : 4;
+    static constexpr int kRingBudget = 70 * 1024;    // per CTA; two CTAs per SM
+    static constexpr int kStagesFit = kRingBudget / (kWarps * kTileSmem);
+    static constexpr int kStages = kStagesFit < 2 ? 2 : (kStagesFit > 6 ? 6 : kStagesFit);
+    static constexpr int kThreads = 32 * kWarps;
+    // common part | per-warp tile descriptors | per-warp rings
+    static __host__ __device__ size_t desc_offset(int B) {
+        return (score_common_bytes(B) + 15) & ~(size_t)15;
+    }
+    static __host__ __device__ size_t ring_offset(int B) {
+        return (desc_offset(B) + (size_t)kWarps * kStages * 16 + 127) & ~(size_t)127;
+    }
+    static __host__ __device__ size_t smem_bytes(int B) {
+        return ring_offset(B) + (size_t)kWarps * kStages * kTileSmem;
+    }
+};
+
+// F8: the rows are the fp8 copy (2D E4M3 bytes + a 16-byte trailer whose
+// first int32 is the row's exponent e).  An ldmatrix of 8 rows x 16 bytes
+// gives lane (g, t) the four channels 4t .. 4t+3 of row g's 16-channel chunk;
+// the hardware converts each pair to f16 (exact), the pairs become the k
+// slots (2t, 2t+1) and (2t+8, 2t+9) of an f16 MMA whose q side takes the same
+// channels, q is converted to f16 (exact for |q| >= 2^-17), and the row's sums
+// are scaled by 2^e.
+template <int D, int NB, bool F8>
+__global__ void __launch_bounds__(RingCfg<D, F8>::kThreads, 2)
+score_ring_kernel(ScoreParams p) {
+    using C = RingCfg<D, F8>;
+    extern __shared__ __align__(16) int smem_i[];
+    int s, e;
+    TileWalker walk = score_setup(p, smem_i, s, e);
+    if (s >= e) return;
+    const int* pt = smem_i;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int B = p.s.B, Hkv = p.s.Hkv, G = p.s.G;
+    const int gq = lane >> 2, tq = lane & 3;
+    uint8_t* ring = reinterpret_cast<uint8_t*>(smem_i) + C::ring_offset(B) +
+                    (size_t)warp * C::kStages * C::kTileSmem;
+    int4* desc = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(smem_i) + C::desc_offset(B)) +
+                 warp * C::kStages;
+    const uint8_t* mbase = F8 ? p.meta8 : reinterpret_cast<const uint8_t*>(p.meta);
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    // ldmatrix row address of this lane: matrices (rows 0-7 | rows 8-15) x (chunk c | c+1)
+    const uint32_t lm_off = (uint32_t)(((lane & 7) + 8 * ((lane >> 3) & 1)) * C::kStride +
+                                       16 * (lane >> 4));
+
+    // copies of one tile's rows into ring stage `stage`; rows past the tile and
+    // rows with a bad page id are zero-filled (their scores are dropped)
+    auto issue = [&](const TileInfo& t, int x0, int stage) {
+        // lane r < 16 resolves row r of the tile: its metadata row, or -1
+        int row_of_lane = -1;
+        if (lane < t.count) {
+            const int ph = pt[x0 + lane];
+            if (ph >= 0 && ph < p.s.NPG) row_of_lane = ph * Hkv + t.unit % Hkv;
+        }
+        const uint32_t dst = ring_s + (uint32_t)(stage * C::kTileSmem);
+#pragma unroll
+        for (int i = 0; i < C::kCopyIters; ++i) {
+            const int id = i * 32 + lane;
+            const int r = id / C::kRowChunks < 16 ? id / C::kRowChunks : 15;
+            const int c = id - r * C::kRowChunks;
+            const int mrow = __shfl_sync(0xffffffffu, row_of_lane, r);
+            if (C::kTileChunks % 32 == 0 || id < C::kTileChunks) {
+                const uint8_t* src =
+                    mbase + (size_t)(mrow >= 0 ? mrow : 0) * C::kRowBytes + 16 * c;
+                cp_async_16(dst + (uint32_t)(r * C::kStride + 16 * c), src, mrow >= 0 ? 16u : 0u);
+            }
+        }
+    };
+
+    // B fragments of [q- | q+] for the current unit: MMA kk covers the 16
+    // channels [16 kk, 16 kk + 16) of the [min | max] row (min pairs with q-)
+    uint32_t qf[D / 8][NB][2];
+    int cur_unit = -1;
+    KeyRange kr;
+
+    auto process = [&](const TileInfo& t, int x0, int stage) {
+        const int b = t.unit / Hkv, g = t.unit % Hkv;
+        if (t.unit != cur_unit) {
+            cur_unit = t.unit;
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int head = nb * 8 + gq;
+                const uint32_t* qw = reinterpret_cast<const uint32_t*>(
+                    p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
+#pragma unroll
+                for (int kk = 0; kk < D / 8; ++kk) {
+                    const bool is_max = 16 * kk >= D;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        // channel pair of k slots (2t, 2t+1) [h = 0] or (2t+8, 2t+9) [h = 1]
+                        const int ch = F8 ? 16 * kk + 4 * tq + 2 * h : 16 * kk + 8 * h + 2 * tq;
+                        const int qc = is_max ? ch - D : ch;
+                        const uint32_t v = head < G ? __ldg(qw + qc / 2) : 0u;
+                        const uint32_t part = is_max ? pos_part(v) : neg_part(v);
+                        qf[kk][nb][h] = F8 ? bf16x2_to_f16x2(part) : part;
+                    }
+                }
+            }
+        }
+        const uint32_t tile = ring_s + (uint32_t)(stage * C::kTileSmem) + lm_off;
+        // two accumulator chains (even and odd MMAs), summed at the end
+        float acc[NB][4], acc2[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[nb][i] = acc2[nb][i] = 0.f;
+        if constexpr (!F8) {
+#pragma unroll
+            for (int kk = 0; kk < D / 8; ++kk) {          // chunks 2kk (k 0-7), 2kk+1 (k 8-15)
+                uint32_t a[4];
+                ldsm_x4(a, tile + 32 * kk);
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    if (kk & 1) mma_bf16_16816(acc2[nb], a, qf[kk][nb][0], qf[kk][nb][1]);
+                    else mma_bf16_16816(acc[nb], a, qf[kk][nb][0], qf[kk][nb][1]);
+                }
+            }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[nb][i] += acc2[nb][i];
+        } else {
+#pragma unroll
+            for (int kp = 0; kp < D / 16; ++kp) {         // chunks 2kp and 2kp+1, one MMA each
+                uint32_t m[4];
+                ldsm_x4(m, tile + 32 * kp);
+                const uint32_t a0[4] = {e4m3x2_to_f16x2(m[0]), e4m3x2_to_f16x2(m[1]),
+                                        e4m3x2_to_f16x2(m[0] >> 16), e4m3x2_to_f16x2(m[1] >> 16)};
+                const uint32_t a1[4] = {e4m3x2_to_f16x2(m[2]), e4m3x2_to_f16x2(m[3]),
+                                        e4m3x2_to_f16x2(m[2] >> 16), e4m3x2_to_f16x2(m[3] >> 16)};
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    mma_f16_16816(acc[nb], a0, qf[2 * kp][nb][0], qf[2 * kp][nb][1]);
+                    mma_f16_16816(acc2[nb], a1, qf[2 * kp + 1][nb][0], qf[2 * kp + 1][nb][1]);
+                }
+            }
+            const uint8_t* rows = ring + stage * C::kTileSmem;
+            const float sc0 = ldexpf(1.f, *reinterpret_cast<const int*>(rows + gq * C::kStride + 2 * D));
+            const float sc8 =
+                ldexpf(1.f, *reinterpret_cast<const int*>(rows + (gq + 8) * C::kStride + 2 * D));
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                acc[nb][0] = (acc[nb][0] + acc2[nb][0]) * sc0;
+                acc[nb][1] = (acc[nb][1] + acc2[nb][1]) * sc0;
+                acc[nb][2] = (acc[nb][2] + acc2[nb][2]) * sc8;
+                acc[nb][3] = (acc[nb][3] + acc2[nb][3]) * sc8;
+            }
+        }
+        int p0, p8;
+        const bool ok0 = row_ok(p, pt, x0, gq, t.count, p0);
+        const bool ok8 = row_ok(p, pt, x0, gq + 8, t.count, p8);
+        score_store<NB>(p, t, acc, ok0, ok8, kr, lane);
+    };
+
+    // this warp's tiles: a contiguous 1/kWarps of the CTA's range, walked once;
+    // copies run kStages - 1 tiles ahead of the processing, and each stage's
+    // tile descriptor waits in shared memory
+    const int ws = s + (int)((long long)(e - s) * warp / C::kWarps);
+    const int we = s + (int)((long long)(e - s) * (warp + 1) / C::kWarps);
+    walk.start(ws, we);
+    auto issue_next = [&](int stage) -> bool {
         TileInfo t;
-        for (int j = 0; walk.next(t); ++j) {
-            if (j % C::kWarps != warp) continue;
-            const int b = t.unit / Hkv, g = t.unit % Hkv;
-            const int x0 = walk.x - t.count - s;           // slice index of row 0
-            // rows g and g+8 of the tile (clamped inside the tile; extra rows are dropped)
-            const int r0 = gq < t.count ? gq : t.count - 1;
-            const int r8 = gq + 8 < t.count ? gq + 8 : t.count - 1;
-            const int p0 = pt[x0 + r0], p8 = pt[x0 + r8];
-            const bool ok0 = p0 >= 0 && p0 < p.s.NPG, ok8 = p8 >= 0 && p8 < p.s.NPG;
-            const char* row0 = reinterpret_cast<const char*>(
-                p.meta + ((size_t)(ok0 ? p0 : 0) * Hkv + g) * 2 * D) + 16 * tq;
-            const char* row8 = reinterpret_cast<const char*>(
-                p.meta + ((size_t)(ok8 ? p8 : 0) * Hkv + g) * 2 * D) + 16 * tq;
-            uint4 xa[C::kKPairs], xb[C::kKPairs];
-    #pragma unroll
-            for (int kp = 0; kp < C::kKPairs; ++kp) {
-                xa[kp] = ld_stream_v4(row0 + 64 * kp);
-                xb[kp] = ld_stream_v4(row8 + 64 * kp);
-            }
-            if (t.unit != cur_unit) {
-                cur_unit = t.unit;
-    #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    const int head = nb * 8 + gq;
-                    const uint32_t* qw = reinterpret_cast<const uint32_t*>(
-                        p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
-    #pragma unroll
-                    for (int kp = 0; kp < C::kKPairs; ++kp) {
-                        // channels ch0 .. ch0+7 of the [min | max] row; min pairs with q-
-                        const int ch0 = 32 * kp + 8 * tq;
-                        const bool is_max = ch0 >= D;
-                        const int qc = is_max ? ch0 - D : ch0;
-    #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const uint32_t v = head < G ? __ldg(qw + qc / 2 + w) : 0u;
-                            qf[kp][nb][w] = is_max ? pos_part(v) : neg_part(v);
-                        }
-                    }
-                }
-            }
-            float acc[NB][4];
-    #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-    #pragma unroll
-            for (int kp = 0; kp < C::kKPairs; ++kp) {
-                const uint32_t a0[4] = {xa[kp].x, xb[kp].x, xa[kp].y, xb[kp].y};
-                const uint32_t a1[4] = {xa[kp].z, xb[kp].z, xa[kp].w, xb[kp].w};
-    #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    mma_bf16_16816(acc[nb], a0, qf[kp][nb][0], qf[kp][nb][1]);
-                    mma_bf16_16816(acc[nb], a1, qf[kp][nb][2], qf[kp][nb][3]);
-                }
-            }
-            // max over the group's heads: this lane holds heads 8nb + 2tq, +1
-            float m0 = -INFINITY, m8 = -INFINITY;
-    #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const int h = nb * 8 + 2 * tq;
-                if (h < G) {
-                    m0 = fmaxf(m0, acc[nb][0]);
-                    m8 = fmaxf(m8, acc[nb][2]);
-                }
-                if (h + 1 < G) {
-                    m0 = fmaxf(m0, acc[nb][1]);
-                    m8 = fmaxf(m8, acc[nb][3]);
-                }
-            }
-            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-            m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
-            m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
-            const int row = tq == 0 ? gq : gq + 8;
-            const bool has = tq < 2 && row < t.count;
-            const bool ok = tq == 0 ? ok0 : ok8;
-            const float v = ok ? (tq == 0 ? m0 : m8) : -INFINITY;
-            if (has) {
-                if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
-                const size_t o = (size_t)t.unit * MP + t.first + row;
-                p.scores_ws[o] = v;
-                if (p.scores_out) p.scores_out[o] = v;
-            }
-            // the unit's key range for the selection (min kept as ~key, so that
-            // both ends merge with atomicMax from a zeroed word), published once
-            // per warp and unit: per-tile atomics on one word serialise in L2
-            const uint32_t key = order_key(v);
-            if (t.unit != kr_unit) {
-                if (lane == 0 && kr_unit >= 0) {
-                    atomicMax(&p.keyrange[kr_unit].x, kr_nmin);
-                    atomicMax(&p.keyrange[kr_unit].y, kr_max);
-                }
-                kr_unit = t.unit;
-                kr_nmin = kr_max = 0u;
-            }
-            kr_nmin = max(kr_nmin, __reduce_max_sync(0xffffffffu, has ? ~key : 0u));
-            kr_max = max(kr_max, __reduce_max_sync(0xffffffffu, has ? key : 0u));
-        }
+        if (!walk.next(t)) return false;
+        const int x0 = walk.x - t.count - s;            // slice index of row 0
+        if (lane == 0) desc[stage] = make_int4(t.unit, t.first, t.count, x0);
+        issue(t, x0, stage);
+        return true;
+    };
+    int pending = 0;
+#pragma unroll
+    for (int k = 0; k < C::kStages - 1; ++k) {
+        if (issue_next(k)) ++pending;
+        cp_async_commit();
     }
-    if (lane == 0 && kr_unit >= 0) {
-        atomicMax(&p.keyrange[kr_unit].x, kr_nmin);
-        atomicMax(&p.keyrange[kr_unit].y, kr_max);
+    for (int stage = 0; pending > 0; stage = stage + 1 == C::kStages ? 0 : stage + 1) {
+        if (issue_next(stage == 0 ? C::kStages - 1 : stage - 1)) ++pending;   // the stage freed last
+        cp_async_commit();
+        cp_async_wait<C::kStages - 1>();
+        __syncwarp();
+        const int4 d = desc[stage];
+        process(TileInfo{d.x, d.y, d.z}, d.w, stage);
+        __syncwarp();
+        --pending;
     }
+    cp_async_wait<0>();
+    kr.flush(p, lane);
+}
+
+// ------------------------------------------------------------ launch
+// Raises a kernel's dynamic shared-memory limit to `bytes` unless done[dev]
+// (the caller's per-kernel record of the largest limit set on each device)
+// already covers it.
+template <typename K>
+cudaError_t ensure_smem(K kern, size_t bytes, size_t (&done)[64]) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && done[dev] >= bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)bytes);
+    if (e == cudaSuccess && dev < 64) done[dev] = bytes;
+    return e;
+}
+
+// Grid: `per_sm` CTAs per SM, or more when the candidates would overflow the
+// CTAs' page-table slices.
+inline unsigned score_grid(const ScoreParams& p, int per_sm) {
+    const long long ub = (long long)p.s.B * p.s.Hkv * p.s.MP;
+    long long grid = (long long)per_sm * device_sm_count();
+    const long long need = (ub + kScorePtCap - 1) / kScorePtCap;
+    if (need > grid) grid = need;
+    return (unsigned)(grid < 1 ? 1 : grid);
+}
+
+template <int D, int NB>
+cudaError_t launch_direct(const ScoreParams& p, cudaStream_t st) {
+    using C = DirectCfg<D, NB>;
+    auto kern = score_direct_kernel<D, NB>;
+    static size_t smem_set[64] = {0};
+    const size_t smem = C::smem_bytes(p.s.B);
+    cudaError_t e = ensure_smem(kern, smem, smem_set);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3(score_grid(p, C::kMinBlocks)), dim3(C::kThreads), smem, st, p);
 }
 
 template <int D, int NB, bool F8>
-cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t st) {
-    using C = ScoreCfg<D, NB>;
-    auto kern = score_kernel<D, NB, F8>;
-    static int attr_done[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)C::smem_bytes(kMaxUnits));
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = 1;
-    }
+cudaError_t launch_ring(const ScoreParams& p, cudaStream_t st) {
+    using C = RingCfg<D, F8>;
+    auto kern = score_ring_kernel<D, NB, F8>;
+    static size_t smem_set[64] = {0};
     const size_t smem = C::smem_bytes(p.s.B);
-    const long long ub = (long long)p.s.B * p.s.Hkv * p.s.MP;
-    long long grid = 2LL * device_sm_count();      // two resident CTAs of 8 warps per SM
-    const long long need = (ub + kScorePtCap - 1) / kScorePtCap;
-    if (need > grid) grid = need;
-    if (grid < 1) grid = 1;
-    return launch_pdl(kern, dim3((unsigned)grid), dim3(C::kThreads), smem, st, p);
+    cudaError_t e = ensure_smem(kern, smem, smem_set);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3(score_grid(p, 2)), dim3(C::kThreads), smem, st, p);
+}
+
+// bf16 metadata: the direct path at D <= 128, the ring at D = 256; the fp8
+// copy: the ring.  Measured on B200: a 256k layer's scoring (D = 128, 262k
+// rows) took 28.5 us direct against 30.2 us in the ring, and 90 against
+// 100 us at four times the rows; the 64k layer (D = 256) took 37.4 us per
+// layer step with the ring against 39.6 us direct; the fp8 copy, 24.7 us in
+// the ring against 29.5 us direct.
+template <int D, int NB>
+cudaError_t launch_score_d(const ScoreParams& p, cudaStream_t st) {
+    if (p.meta8) return launch_ring<D, NB, true>(p, st);
+    if constexpr (D == 256) return launch_ring<D, NB, false>(p, st);
+    else return launch_direct<D, NB>(p, st);
 }
 
 }  // namespace
@@ -518,18 +629,12 @@ cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t st) {
 cudaError_t launch_score(const ScoreParams& p, cudaStream_t st) {
     const int nb = p.s.G > 8 ? 2 : 1;
     switch (p.s.D * 10 + nb) {
-        case 641: return p.meta8 ? launch_score_t<64, 1, true>(p, st)
-                          : launch_score_t<64, 1, false>(p, st);
-        case 642: return p.meta8 ? launch_score_t<64, 2, true>(p, st)
-                          : launch_score_t<64, 2, false>(p, st);
-        case 1281: return p.meta8 ? launch_score_t<128, 1, true>(p, st)
-                          : launch_score_t<128, 1, false>(p, st);
-        case 1282: return p.meta8 ? launch_score_t<128, 2, true>(p, st)
-                          : launch_score_t<128, 2, false>(p, st);
-        case 2561: return p.meta8 ? launch_score_t<256, 1, true>(p, st)
-                          : launch_score_t<256, 1, false>(p, st);
-        case 2562: return p.meta8 ? launch_score_t<256, 2, true>(p, st)
-                          : launch_score_t<256, 2, false>(p, st);
+        case 641: return launch_score_d<64, 1>(p, st);
+        case 642: return launch_score_d<64, 2>(p, st);
+        case 1281: return launch_score_d<128, 1>(p, st);
+        case 1282: return launch_score_d<128, 2>(p, st);
+        case 2561: return launch_score_d<256, 1>(p, st);
+        case 2562: return launch_score_d<256, 2>(p, st);
         default: return cudaErrorInvalidValue;
     }
 }
