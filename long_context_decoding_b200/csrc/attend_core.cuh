@@ -112,6 +112,21 @@ __device__ __forceinline__ void load_page(uint32_t buf, const uint16_t* kt, cons
     }
 }
 
+// The same for one of the two tiles (K or V) of a page.
+template <int D>
+__device__ __forceinline__ void load_half(uint32_t buf, const uint16_t* t, int rows_valid,
+                                          int lane) {
+    constexpr int kChunksPerRow = D / 8;
+    constexpr int kChunks = 16 * kChunksPerRow;
+#pragma unroll
+    for (int i = 0; i < kChunks / 32; ++i) {
+        const int idx = i * 32 + lane;
+        const int r = idx / kChunksPerRow, c16 = idx % kChunksPerRow;
+        const uint32_t off = (c16 >> 3) * 2048 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+        cp_async_16(buf + off, t + (size_t)r * D + c16 * 8, r < rows_valid ? 16u : 0u);
+    }
+}
+
 // Shared-memory footprint of the core for W warps with BUFS page buffers.
 template <int D, int NB, int W, int BUFS>
 struct TileCfg {
@@ -180,113 +195,147 @@ __device__ void attend_unit(const AttendArgs& A, int u, int L, const int2* items
             o[mb][nb][0] = o[mb][nb][1] = o[mb][nb][2] = o[mb][nb][3] = 0.f;
     }
 
-    // this warp's items of the segment: a + warp, a + warp + W, ...
-    auto issue = [&](long long x, int slot) {
-        const int2 it = items[x - s];
-        if (it.x >= 0) {
-            const int page = it.y >> 2;
-            const size_t tile = ((size_t)it.x * Hkv + g) * kPage * D;
-            const int rows = L - page * kPage < kPage ? L - page * kPage : kPage;
-            load_page<D>(wbuf + (uint32_t)(slot * T::kPageBytes), A.k_cache + tile,
-                         A.v_cache + tile, rows, lane);
+    // ---- S^T = K Q^T for the page in the buffer at kbase, the mask and the
+    // online softmax (exp2 domain); leaves P^T as B fragments in pb
+    auto qk_softmax = [&](uint32_t kbase, int page, int mask, uint32_t (&pb)[NB][2]) {
+        float sacc[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+            sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < T::kMB; ++kb) {
+            const int chunk = 2 * kb + k_half;
+            const uint32_t addr =
+                kbase + (chunk >> 3) * 2048 + k_tok * 128 + (((chunk & 7) ^ ri) << 4);
+            uint32_t af[4];
+            ldsm_x4(af, addr);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+                mma_bf16_16816(sacc[nb], af, qf[kb][nb][0], qf[kb][nb][1]);
         }
-        cp_async_commit();
+        const int t0 = page * kPage + gq, t1 = t0 + 8;
+        const bool f0 = t0 < Pe || t0 >= Lw, f1 = t1 < Pe || t1 >= Lw;
+        const bool in0 = t0 < L && (mask == kMaskAll || (mask == kMaskFixed) == f0);
+        const bool in1 = t1 < L && (mask == kMaskAll || (mask == kMaskFixed) == f1);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            const float s00 = in0 ? sacc[nb][0] * sl2 : -INFINITY;
+            const float s01 = in0 ? sacc[nb][1] * sl2 : -INFINITY;
+            const float s10 = in1 ? sacc[nb][2] * sl2 : -INFINITY;
+            const float s11 = in1 ? sacc[nb][3] * sl2 : -INFINITY;
+            float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+#pragma unroll
+            for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+            }
+            const float mn0 = fmaxf(m[nb][0], mx0), mn1 = fmaxf(m[nb][1], mx1);
+            const float base0 = mn0 == -INFINITY ? 0.f : mn0;
+            const float base1 = mn1 == -INFINITY ? 0.f : mn1;
+            const float al0 = ex2(m[nb][0] - base0), al1 = ex2(m[nb][1] - base1);
+            const uint32_t P0 = pack_bf16x2(ex2(s00 - base0), ex2(s01 - base1));
+            const uint32_t P1 = pack_bf16x2(ex2(s10 - base0), ex2(s11 - base1));
+            l[nb][0] = l[nb][0] * al0 + bf16_lo(P0) + bf16_lo(P1);
+            l[nb][1] = l[nb][1] * al1 + bf16_hi(P0) + bf16_hi(P1);
+            m[nb][0] = mn0;
+            m[nb][1] = mn1;
+#pragma unroll
+            for (int mb = 0; mb < T::kMB; ++mb) {
+                o[mb][nb][0] *= al0;
+                o[mb][nb][1] *= al1;
+                o[mb][nb][2] *= al0;
+                o[mb][nb][3] *= al1;
+            }
+            pb[nb][0] = movmatrix_trans(P0);
+            pb[nb][1] = movmatrix_trans(P1);
+        }
     };
-    long long x = a + warp;
-    int slot = 0;
-    if (x < bnd) issue(x, 0);
-    for (; x < bnd; x += W) {
-        const long long xn = x + W;
-        if (BUFS == 2) {
+    // ---- O^T += V^T P^T for the page in the buffer at vbase
+    auto pv = [&](uint32_t vbase, const uint32_t (&pb)[NB][2]) {
+#pragma unroll
+        for (int mb = 0; mb < T::kMB; ++mb) {
+            const int chunk = 2 * mb + v_half;
+            const uint32_t addr =
+                vbase + (chunk >> 3) * 2048 + v_tok * 128 + (((chunk & 7) ^ ri) << 4);
+            uint32_t af[4];
+            ldsm_x4_trans(af, addr);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+                mma_bf16_16816(o[mb][nb], af, pb[nb][0], pb[nb][1]);
+        }
+    };
+
+    // this warp's items of the segment: a + warp, a + warp + W, ...
+    if constexpr (BUFS == 2) {
+        auto issue = [&](long long x, int slot) {
+            const int2 it = items[x - s];
+            if (it.x >= 0) {
+                const int page = it.y >> 2;
+                const size_t tile = ((size_t)it.x * Hkv + g) * kPage * D;
+                const int rows = L - page * kPage < kPage ? L - page * kPage : kPage;
+                load_page<D>(wbuf + (uint32_t)(slot * T::kPageBytes), A.k_cache + tile,
+                             A.v_cache + tile, rows, lane);
+            }
+            cp_async_commit();
+        };
+        long long x = a + warp;
+        int slot = 0;
+        if (x < bnd) issue(x, 0);
+        for (; x < bnd; x += W) {
+            const long long xn = x + W;
             if (xn < bnd) {
                 issue(xn, slot ^ 1);
                 cp_async_wait<1>();
             } else {
                 cp_async_wait<0>();
             }
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncwarp();
-        const int2 it = items[x - s];
-        if (it.x >= 0) {
-            const int page = it.y >> 2;
-            const int mask = it.y & 3;
-            const uint32_t kbase = wbuf + (uint32_t)(slot * T::kPageBytes);
-            const uint32_t vbase = kbase + T::kHalf;
-            // ---- S^T = K Q^T
-            float sacc[NB][4];
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb)
-                sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
-#pragma unroll
-            for (int kb = 0; kb < T::kMB; ++kb) {
-                const int chunk = 2 * kb + k_half;
-                const uint32_t addr =
-                    kbase + (chunk >> 3) * 2048 + k_tok * 128 + (((chunk & 7) ^ ri) << 4);
-                uint32_t af[4];
-                ldsm_x4(af, addr);
-#pragma unroll
-                for (int nb = 0; nb < NB; ++nb)
-                    mma_bf16_16816(sacc[nb], af, qf[kb][nb][0], qf[kb][nb][1]);
+            __syncwarp();
+            const int2 it = items[x - s];
+            if (it.x >= 0) {
+                const uint32_t kbase = wbuf + (uint32_t)(slot * T::kPageBytes);
+                uint32_t pb[NB][2];
+                qk_softmax(kbase, it.y >> 2, it.y & 3, pb);
+                pv(kbase + T::kHalf, pb);
             }
-            // ---- mask and online softmax (exp2 domain)
-            const int t0 = page * kPage + gq, t1 = t0 + 8;
-            const bool f0 = t0 < Pe || t0 >= Lw, f1 = t1 < Pe || t1 >= Lw;
-            const bool in0 = t0 < L && (mask == kMaskAll || (mask == kMaskFixed) == f0);
-            const bool in1 = t1 < L && (mask == kMaskAll || (mask == kMaskFixed) == f1);
-            uint32_t pb[NB][2];
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const float s00 = in0 ? sacc[nb][0] * sl2 : -INFINITY;
-                const float s01 = in0 ? sacc[nb][1] * sl2 : -INFINITY;
-                const float s10 = in1 ? sacc[nb][2] * sl2 : -INFINITY;
-                const float s11 = in1 ? sacc[nb][3] * sl2 : -INFINITY;
-                float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
-#pragma unroll
-                for (int o2 = 4; o2 < 32; o2 <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
-                }
-                const float mn0 = fmaxf(m[nb][0], mx0), mn1 = fmaxf(m[nb][1], mx1);
-                const float base0 = mn0 == -INFINITY ? 0.f : mn0;
-                const float base1 = mn1 == -INFINITY ? 0.f : mn1;
-                const float al0 = ex2(m[nb][0] - base0), al1 = ex2(m[nb][1] - base1);
-                const uint32_t P0 = pack_bf16x2(ex2(s00 - base0), ex2(s01 - base1));
-                const uint32_t P1 = pack_bf16x2(ex2(s10 - base0), ex2(s11 - base1));
-                l[nb][0] = l[nb][0] * al0 + bf16_lo(P0) + bf16_lo(P1);
-                l[nb][1] = l[nb][1] * al1 + bf16_hi(P0) + bf16_hi(P1);
-                m[nb][0] = mn0;
-                m[nb][1] = mn1;
-#pragma unroll
-                for (int mb = 0; mb < T::kMB; ++mb) {
-                    o[mb][nb][0] *= al0;
-                    o[mb][nb][1] *= al1;
-                    o[mb][nb][2] *= al0;
-                    o[mb][nb][3] *= al1;
-                }
-                pb[nb][0] = movmatrix_trans(P0);
-                pb[nb][1] = movmatrix_trans(P1);
-            }
-            // ---- O^T += V^T P^T
-#pragma unroll
-            for (int mb = 0; mb < T::kMB; ++mb) {
-                const int chunk = 2 * mb + v_half;
-                const uint32_t addr =
-                    vbase + (chunk >> 3) * 2048 + v_tok * 128 + (((chunk & 7) ^ ri) << 4);
-                uint32_t af[4];
-                ldsm_x4_trans(af, addr);
-#pragma unroll
-                for (int nb = 0; nb < NB; ++nb)
-                    mma_bf16_16816(o[mb][nb], af, pb[nb][0], pb[nb][1]);
-            }
-        }
-        __syncwarp();                 // the buffer is refilled next
-        if (BUFS == 1) {
-            if (xn < bnd) issue(xn, 0);
-        } else {
+            __syncwarp();                 // the buffer is refilled next
             slot ^= 1;
         }
+    } else {
+        // one buffer: its K and V halves are refilled separately, so that the
+        // next page's K streams in during this page's P V and its V during the
+        // next Q K (one cp.async group per half, always committed)
+        auto issue_half = [&](long long x, int half) {
+            if (x < bnd) {
+                const int2 it = items[x - s];
+                if (it.x >= 0) {
+                    const int page = it.y >> 2;
+                    const size_t tile = ((size_t)it.x * Hkv + g) * kPage * D;
+                    const int rows = L - page * kPage < kPage ? L - page * kPage : kPage;
+                    load_half<D>(wbuf + (uint32_t)(half * T::kHalf),
+                                 (half ? A.v_cache : A.k_cache) + tile, rows, lane);
+                }
+            }
+            cp_async_commit();
+        };
+        long long x = a + warp;
+        issue_half(x, 0);
+        issue_half(x, 1);
+        for (; x < bnd; x += W) {
+            const long long xn = x + W;
+            const int2 it = items[x - s];
+            uint32_t pb[NB][2];
+            cp_async_wait<1>();           // this page's K
+            __syncwarp();
+            if (it.x >= 0) qk_softmax(wbuf, it.y >> 2, it.y & 3, pb);
+            __syncwarp();                 // K is refilled next
+            issue_half(xn, 0);
+            cp_async_wait<1>();           // this page's V
+            __syncwarp();
+            if (it.x >= 0) pv(wbuf + T::kHalf, pb);
+            __syncwarp();                 // V is refilled next
+            issue_half(xn, 1);
+        }
+        cp_async_wait<0>();
     }
 
     // ---- merge the warps of this CTA (Ow aliases the page buffers)
