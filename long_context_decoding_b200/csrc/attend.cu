@@ -35,14 +35,17 @@ namespace csa {
 namespace {
 
 constexpr int kFusedUnits = 32;            // units the fused path serves
-constexpr int kFusedItems = kClCap / kCl;  // pages of one CTA's share (2048)
+constexpr int kFusedItems = kClCap / kCl;  // work items of one CTA: its share of a unit's
+                                           // selected pages (2048), or its prefix/window slice
 constexpr int kFusedMinItems = 4 * 8;      // prefix/window pages per CTA, at least (16 measured slower)
 
 template <int D, int NB>
 struct FusedCfg {
     static constexpr int kWarps = 8;                    // == kClThreads / 32
-    static constexpr int kBufs = 1;
-    using Tile = TileCfg<D, NB, kWarps, kBufs>;
+    // K/V tile slots per warp: two keep two CTAs per SM at D <= 128 (three
+    // slots, with smaller item lists, measured no faster)
+    static constexpr int kHalves = 2;
+    using Tile = TileCfg<D, NB, kWarps, kHalves>;
     static constexpr size_t kItems = (size_t)kFusedItems * 8;
     static constexpr size_t kUnits = (size_t)(kFusedUnits + 1) * 4 + (size_t)kFusedUnits * 4;
     static constexpr size_t kSmem = 1024 /* alignment slack */ + Tile::kStageArea + Tile::kMl +
@@ -136,7 +139,7 @@ __global__ void __cluster_dims__(kCl, 1, 1)
             const long long a = s > uoff[u] ? s : uoff[u];
             const long long bnd = e < uoff[u + 1] ? e : uoff[u + 1];
             if (a >= bnd) continue;
-            attend_unit<D, NB, C::kWarps, C::kBufs>(A, u, ulen[u], items, s, a, bnd, stages, ms,
+            attend_unit<D, NB, C::kWarps, C::kHalves>(A, u, ulen[u], items, s, a, bnd, stages, ms,
                                                      ls, p.partials + ((size_t)c0 + u) * rs);
             const int first = cta_of(uoff[u], T0, n_cta);
             if (c0 == first && tid == 0)
@@ -200,7 +203,7 @@ __global__ void __cluster_dims__(kCl, 1, 1)
         items[j] = make_int2(phys, page * 4 + kMaskRest);
     }
     __syncthreads();
-    attend_unit<D, NB, C::kWarps, C::kBufs>(A, u, L, items, 0, 0, cnt, stages, ms, ls,
+    attend_unit<D, NB, C::kWarps, C::kHalves>(A, u, L, items, 0, 0, cnt, stages, ms, ls,
                                              p.partials + p.phase_floats +
                                                  ((size_t)kCl * u + rank) * rs);
 }
@@ -234,18 +237,28 @@ bool fused_eligible(const Shape& s, int prefix, int window, int k_pages) {
     return k_pages > 0 && (long long)s.B * s.Hkv <= kFusedUnits && n_max <= kClCap;
 }
 
-// CTAs of the prefix/window role: what stays of the resident capacity beside
-// the selection clusters, at least enough that no slice exceeds the item
-// capacity, and a whole number of clusters.
-int fused_phase0_ctas(const Shape& s) {
+// CTAs of the prefix/window role for a call: what stays of the resident
+// capacity beside the selection clusters, at least enough that no slice
+// exceeds the item capacity (every unit's fixed list holds at most
+// ceil(prefix / 16) + ceil(window / 16) + 2 pages), and a whole number of
+// clusters.
+int fused_phase0_ctas(const Shape& s, long long prefix, long long window) {
     const long long units = (long long)s.B * s.Hkv;
     const int per_sm = (s.D <= 128 && s.G <= 8) ? 2 : 1;
     long long n0 = (long long)per_sm * device_sm_count() - kCl * units;
-    const long long cap = (units * (s.MP + 2) + kFusedItems - 1) / kFusedItems;
+    long long fixed = (prefix + kPage - 1) / kPage + (window + kPage - 1) / kPage + 2;
+    if (fixed > (long long)s.MP + 2) fixed = (long long)s.MP + 2;
+    const long long cap = (units * fixed + kFusedItems - 1) / kFusedItems;
     if (n0 < cap) n0 = cap;
     if (n0 < kCl) n0 = kCl;
     n0 = (n0 + kCl - 1) / kCl * kCl;
     return (int)(n0 < (1ll << 30) ? n0 : (1ll << 30));
+}
+
+// The most any call of the shape needs (for the workspace).
+int fused_phase0_ctas(const Shape& s) {
+    const long long all = (long long)s.MP * kPage;
+    return fused_phase0_ctas(s, all, all);
 }
 
 cudaError_t launch_fused(const FusedParams& p, cudaStream_t st) {

@@ -12,10 +12,14 @@
 // combine kernel merges with the unit's other records.
 //
 // Every warp streams its own pages (round-robin over the slice) with 16-byte
-// cp.async copies into BUFS private page buffers, laid out with the 128-byte
-// XOR swizzle (16-byte chunk c of token row r at c ^ (r & 7)) so that ldmatrix
+// cp.async copies into a private ring of HALVES slots, each holding the K or
+// the V tile of one page (16 tokens x D), laid out with the 128-byte XOR
+// swizzle (16-byte chunk c of token row r at c ^ (r & 7)) so that ldmatrix
 // reads them without bank conflicts; rows past the end of the sequence are
-// zero-filled by the copy itself.  Per page: S^T = K Q^T (16 tokens x 8
+// zero-filled by the copy itself.  The tiles are consumed in the order K0,
+// V0, K1, V1, ... and a slot is refilled with the tile HALVES places ahead
+// as soon as its tile has been used, so HALVES - 1 tiles stay in flight while
+// the warp computes (the attention is bound by the bytes in flight).  Per page: S^T = K Q^T (16 tokens x 8
 // heads, mma.sync m16n8k16 with K fragments from ldmatrix and Q^T fragments
 // in registers), the token mask, the fp32 online softmax in the exp2 domain,
 // P turned into the B operand by movmatrix, and O^T += V^T P^T with
@@ -94,25 +98,8 @@ __host__ __device__ __forceinline__ size_t record_stride(int G, int D) {
     return ((size_t)G * D + 2 * G + 3) & ~(size_t)3;
 }
 
-// Issues the cp.async copies of one page's K and V tiles (16 tokens x D) into
-// a swizzled buffer; token rows >= rows_valid are zero-filled.
-template <int D>
-__device__ __forceinline__ void load_page(uint32_t buf, const uint16_t* kt, const uint16_t* vt,
-                                          int rows_valid, int lane) {
-    constexpr int kChunksPerRow = D / 8;
-    constexpr int kChunks = 16 * kChunksPerRow;
-#pragma unroll
-    for (int i = 0; i < kChunks / 32; ++i) {
-        const int idx = i * 32 + lane;
-        const int r = idx / kChunksPerRow, c16 = idx % kChunksPerRow;
-        const uint32_t off = (c16 >> 3) * 2048 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-        const uint32_t n = r < rows_valid ? 16u : 0u;
-        cp_async_16(buf + off, kt + (size_t)r * D + c16 * 8, n);
-        cp_async_16(buf + 32 * D + off, vt + (size_t)r * D + c16 * 8, n);
-    }
-}
-
-// The same for one of the two tiles (K or V) of a page.
+// Issues the cp.async copies of one tile (K or V) of a page (16 tokens x D)
+// into a swizzled slot; token rows >= rows_valid are zero-filled.
 template <int D>
 __device__ __forceinline__ void load_half(uint32_t buf, const uint16_t* t, int rows_valid,
                                           int lane) {
@@ -127,14 +114,14 @@ __device__ __forceinline__ void load_half(uint32_t buf, const uint16_t* t, int r
     }
 }
 
-// Shared-memory footprint of the core for W warps with BUFS page buffers.
-template <int D, int NB, int W, int BUFS>
+// Shared-memory footprint of the core for W warps with HALVES tile slots each.
+template <int D, int NB, int W, int HALVES>
 struct TileCfg {
+    static_assert(HALVES >= 2, "a page's K and V tiles both fit the ring");
     static constexpr int kHalf = 32 * D;                // bytes of one page's K (or V) tile
-    static constexpr int kPageBytes = 2 * kHalf;
     static constexpr int kHeads = 8 * NB;               // query heads per CTA (padded)
     static constexpr int kMB = D / 16;                  // 16-channel blocks
-    static constexpr size_t kStageArea = (size_t)W * BUFS * kPageBytes;
+    static constexpr size_t kStageArea = (size_t)W * HALVES * kHalf;
     static constexpr size_t kOw = (size_t)W * kHeads * D * 4;   // aliases the stage area
     static_assert(kOw <= kStageArea, "the merge buffer lives in the stage area");
     static constexpr size_t kMl = (size_t)2 * W * kHeads * 4;  // per-warp m and l
@@ -153,11 +140,11 @@ struct AttendArgs {
 // (physical page or -1 to skip, page * 4 + mask)) and writes the CTA's
 // partial record of the unit to rec.  Called by all W warps of the CTA; the
 // stage area, ms and ls are free on entry and again on return.
-template <int D, int NB, int W, int BUFS>
+template <int D, int NB, int W, int HALVES>
 __device__ void attend_unit(const AttendArgs& A, int u, int L, const int2* items, long long s,
                             long long a, long long bnd, uint8_t* stages, float* ms, float* ls,
                             float* rec) {
-    using T = TileCfg<D, NB, W, BUFS>;
+    using T = TileCfg<D, NB, W, HALVES>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
     const int mi = lane >> 3, ri = lane & 7;
@@ -169,7 +156,7 @@ __device__ void attend_unit(const AttendArgs& A, int u, int L, const int2* items
     const int b = u / Hkv, g = u % Hkv;
     const SeqGeom sg = seq_geom(L, A.prefix, A.window);
     const int Pe = sg.Pe, Lw = L - sg.We;
-    const uint32_t wbuf = smem_u32(stages) + (uint32_t)(warp * BUFS * T::kPageBytes);
+    const uint32_t wbuf = smem_u32(stages) + (uint32_t)(warp * HALVES * T::kHalf);
     float* Ow = reinterpret_cast<float*>(stages);      // reused after the page loop
 
     // Q^T as the B operand: b0 = q[head][16kb + 2tq, +1], b1 = +8
@@ -265,78 +252,40 @@ __device__ void attend_unit(const AttendArgs& A, int u, int L, const int2* items
         }
     };
 
-    // this warp's items of the segment: a + warp, a + warp + W, ...
-    if constexpr (BUFS == 2) {
-        auto issue = [&](long long x, int slot) {
-            const int2 it = items[x - s];
+    // this warp's items of the segment: a + warp, a + warp + W, ...; tile h of
+    // the warp is the K (h even) or V (h odd) tile of item a + warp + (h / 2) W
+    const long long first = a + warp;
+    const int n_items = first < bnd ? (int)((bnd - first + W - 1) / W) : 0;
+    auto issue = [&](int h, uint32_t slot) {   // one cp.async group per tile, always
+        if (h < 2 * n_items) {
+            const int2 it = items[first + (long long)(h >> 1) * W - s];
             if (it.x >= 0) {
                 const int page = it.y >> 2;
                 const size_t tile = ((size_t)it.x * Hkv + g) * kPage * D;
                 const int rows = L - page * kPage < kPage ? L - page * kPage : kPage;
-                load_page<D>(wbuf + (uint32_t)(slot * T::kPageBytes), A.k_cache + tile,
-                             A.v_cache + tile, rows, lane);
+                load_half<D>(slot, ((h & 1) ? A.v_cache : A.k_cache) + tile, rows, lane);
             }
-            cp_async_commit();
-        };
-        long long x = a + warp;
-        int slot = 0;
-        if (x < bnd) issue(x, 0);
-        for (; x < bnd; x += W) {
-            const long long xn = x + W;
-            if (xn < bnd) {
-                issue(xn, slot ^ 1);
-                cp_async_wait<1>();
-            } else {
-                cp_async_wait<0>();
-            }
-            __syncwarp();
-            const int2 it = items[x - s];
-            if (it.x >= 0) {
-                const uint32_t kbase = wbuf + (uint32_t)(slot * T::kPageBytes);
-                uint32_t pb[NB][2];
-                qk_softmax(kbase, it.y >> 2, it.y & 3, pb);
-                pv(kbase + T::kHalf, pb);
-            }
-            __syncwarp();                 // the buffer is refilled next
-            slot ^= 1;
         }
-    } else {
-        // one buffer: its K and V halves are refilled separately, so that the
-        // next page's K streams in during this page's P V and its V during the
-        // next Q K (one cp.async group per half, always committed)
-        auto issue_half = [&](long long x, int half) {
-            if (x < bnd) {
-                const int2 it = items[x - s];
-                if (it.x >= 0) {
-                    const int page = it.y >> 2;
-                    const size_t tile = ((size_t)it.x * Hkv + g) * kPage * D;
-                    const int rows = L - page * kPage < kPage ? L - page * kPage : kPage;
-                    load_half<D>(wbuf + (uint32_t)(half * T::kHalf),
-                                 (half ? A.v_cache : A.k_cache) + tile, rows, lane);
-                }
-            }
-            cp_async_commit();
-        };
-        long long x = a + warp;
-        issue_half(x, 0);
-        issue_half(x, 1);
-        for (; x < bnd; x += W) {
-            const long long xn = x + W;
-            const int2 it = items[x - s];
-            uint32_t pb[NB][2];
-            cp_async_wait<1>();           // this page's K
-            __syncwarp();
-            if (it.x >= 0) qk_softmax(wbuf, it.y >> 2, it.y & 3, pb);
-            __syncwarp();                 // K is refilled next
-            issue_half(xn, 0);
-            cp_async_wait<1>();           // this page's V
-            __syncwarp();
-            if (it.x >= 0) pv(wbuf + T::kHalf, pb);
-            __syncwarp();                 // V is refilled next
-            issue_half(xn, 1);
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int h = 0; h < HALVES; ++h) issue(h, wbuf + (uint32_t)(h * T::kHalf));
+    uint32_t pb[NB][2];
+    int slot = 0;
+    for (int h = 0; h < 2 * n_items; ++h) {
+        cp_async_wait<HALVES - 1>();   // tile h has landed
+        __syncwarp();
+        const uint32_t buf = wbuf + (uint32_t)(slot * T::kHalf);
+        const int2 it = items[first + (long long)(h >> 1) * W - s];
+        if (it.x >= 0) {
+            if (h & 1) pv(buf, pb);
+            else qk_softmax(buf, it.y >> 2, it.y & 3, pb);
         }
-        cp_async_wait<0>();
+        __syncwarp();                  // the slot is refilled next
+        issue(h + HALVES, buf);
+        slot = slot + 1 == HALVES ? 0 : slot + 1;
     }
+    cp_async_wait<0>();
 
     // ---- merge the warps of this CTA (Ow aliases the page buffers)
     __syncthreads();

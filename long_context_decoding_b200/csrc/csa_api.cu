@@ -417,7 +417,7 @@ static int sparse_attention_common(const csa_dims* d, const void* q, const void*
         fp.sel = sel_pages;
         fp.n_sel = n_sel;
         fp.keyrange = sp.keyrange;
-        fp.n0 = fused_phase0_ctas(s);
+        fp.n0 = fused_phase0_ctas(s, prefix, window);
         return launch_status(launch_fused(fp, st));
     }
     SelectParams lp;

@@ -50,8 +50,8 @@ struct DecCfg {
     // so that three fit beside a CTA of the selection kernel when both are
     // resident (16 heads would spill at that bound)
     static constexpr int kMinBlocks = D == 256 ? 1 : (NB == 1 ? 4 : 3);
-    static constexpr int kBufs = D == 256 ? 1 : 2;      // page buffers per warp
-    using Tile = TileCfg<D, NB, kWarps, kBufs>;
+    static constexpr int kHalves = D == 256 ? 2 : 4;    // K/V tile slots per warp
+    using Tile = TileCfg<D, NB, kWarps, kHalves>;
     static constexpr size_t kStageArea = Tile::kStageArea;
     static constexpr size_t kMl = Tile::kMl;
     static constexpr int kHeads = Tile::kHeads;
@@ -297,7 +297,7 @@ decode_kernel(DecodeParams p) {
             const long long a = s > uoff[u] ? s : uoff[u];
             const long long bnd = e < uoff[u + 1] ? e : uoff[u + 1];
             if (a >= bnd) continue;
-            attend_unit<D, NB, C::kWarps, C::kBufs>(A, u, uinfo[u].x, items, s, a, bnd, stages, ms,
+            attend_unit<D, NB, C::kWarps, C::kHalves>(A, u, uinfo[u].x, items, s, a, bnd, stages, ms,
                                                      ls, region + ((size_t)blockIdx.x + u) * rs);
             const int first_cta = cta_of(uoff[u], T, n_cta);
             if (blockIdx.x == first_cta && tid == 0)

@@ -108,6 +108,7 @@ struct FusedParams {
 };
 bool fused_eligible(const Shape& s, int prefix, int window, int k_pages);
 int fused_phase0_ctas(const Shape& s);
+int fused_phase0_ctas(const Shape& s, long long prefix, long long window);
 cudaError_t launch_fused(const FusedParams& p, cudaStream_t st);
 
 // Kind of the last kernel-launching call issued on a stream (host side).
