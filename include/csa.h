@@ -251,6 +251,59 @@ int csa_sparse_attention_fp8(const csa_dims *d, const void *q, const void *k_cac
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * ------------------------------------------------- context parallelism
+ * One layer's decode with every sequence's pages split over R ranks (each
+ * rank holds the pages [page_lo, page_hi) of every sequence in its own
+ * cache; rank 0 holds the prefix, the last rank the window), with one
+ * exchange step: each rank scores its candidate pages (csa_score_select with
+ * budget 0 and scores_out), the ranks all-gather the score arrays and
+ * concatenate them along the page axis, every rank selects the global top-k
+ * with csa_select_scores (the same pages csa_score_select would select on
+ * one GPU), keeps its own pages with csa_shard_selection, attends over them
+ * and its share of prefix/window with csa_decode, and the ranks all-gather
+ * (out, lse) and merge them with csa_merge_attention.  The exact top-k of the
+ * union is the top-k of the concatenated scores, and the attention over a
+ * union of disjoint token sets is the log-sum-exp merge of the attentions
+ * over the parts, so the result is the single-GPU one up to the bf16 rounding
+ * of the parts' outputs.
+ */
+
+/*
+ * Top-k page selection over caller-provided Quest scores: scores is fp32
+ * [B][Hkv][max_pages_per_seq] (read only; entries outside each unit's
+ * candidate range [c_lo, c_hi), as seq_lens, prefix and window define it,
+ * are ignored), k = budget_tokens / 16, ties to the lower page, output
+ * ascending, exactly as csa_score_select.  Uses the workspace of `d`.
+ */
+int csa_select_scores(const csa_dims *d, const float *scores, const int32_t *seq_lens,
+                      int prefix, int window, int budget_tokens, int32_t *sel_pages,
+                      int32_t *n_sel, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The pages of a selection that fall in [page_lo, page_hi), as pages of the
+ * shard: sel_local[b][g][j] = sel_pages[b][g][i] - page_lo for the selected
+ * pages in range, in ascending order, and n_sel_local[b][g] their count.
+ * sel_pages/n_sel as csa_score_select writes them for dims d (ascending,
+ * n_sel <= d->max_sel); sel_local is int32 [B][Hkv][max_sel_local] with
+ * max_sel_local >= d->max_sel (else CSA_ERR_INVALID_ARG).
+ */
+int csa_shard_selection(const csa_dims *d, const int32_t *sel_pages, const int32_t *n_sel,
+                        int page_lo, int page_hi, int max_sel_local, int32_t *sel_local,
+                        int32_t *n_sel_local, void *stream);
+
+/*
+ * Log-sum-exp merge of `parts` partial attention results over disjoint token
+ * sets: out_parts bf16 [parts][batch][q_heads][head_dim], lse_parts fp32
+ * [parts][batch][q_heads] (natural log; -inf for a part that attended no
+ * token) -> out bf16 [batch][q_heads][head_dim] = sum_r e^(lse_r - lse)
+ * out_r (fp32, rounded to nearest even) and lse fp32 [batch][q_heads] =
+ * log sum_r e^(lse_r) (NULL to skip).  A head no part attended gets out 0 and
+ * lse -inf.  head_dim is 64, 128 or 256; 1 <= parts <= 64.
+ */
+int csa_merge_attention(int parts, int batch, int q_heads, int head_dim, const void *out_parts,
+                        const float *lse_parts, void *out, float *lse, void *stream);
+
+/*
  * csa_decode for callers that cannot allocate device memory.  The paper has
  * no counterpart to this entry point; it exists for deployment: a plugin
  * hosted inside another runtime that owns every device buffer, or a server

@@ -27,7 +27,8 @@ DEVFLAG_TIMEOUT = 8
 EXPORTS = ("csa_version", "csa_status_string", "csa_workspace_size", "csa_workspace_init",
            "csa_meta_update", "csa_score_select", "csa_decode", "csa_decode_full",
            "csa_get_device_status", "csa_decode_noalloc", "csa_sparse_attention",
-           "csa_meta_update_fp8", "csa_score_select_fp8", "csa_sparse_attention_fp8")
+           "csa_meta_update_fp8", "csa_score_select_fp8", "csa_sparse_attention_fp8",
+           "csa_select_scores", "csa_shard_selection", "csa_merge_attention")
 
 
 class CsaError(RuntimeError):
@@ -82,9 +83,13 @@ def lib() -> ctypes.CDLL:
         L.csa_score_select_fp8.argtypes = [D, P, P, P, P, I, I, I, P, P, P, P, Z, P]
         L.csa_sparse_attention_fp8.argtypes = [D, P, P, P, P, P, P, I, I, I, ctypes.c_float, P,
                                                P, P, P, P, Z, P]
+        L.csa_select_scores.argtypes = [D, P, P, I, I, I, P, P, P, Z, P]
+        L.csa_shard_selection.argtypes = [D, P, P, I, I, I, P, P, P]
+        L.csa_merge_attention.argtypes = [I, I, I, I, P, P, P, P, P]
         for f in ("csa_workspace_init", "csa_meta_update", "csa_score_select", "csa_decode",
                   "csa_decode_full", "csa_get_device_status", "csa_sparse_attention",
-                  "csa_meta_update_fp8", "csa_score_select_fp8", "csa_sparse_attention_fp8"):
+                  "csa_meta_update_fp8", "csa_score_select_fp8", "csa_sparse_attention_fp8",
+                  "csa_select_scores", "csa_shard_selection", "csa_merge_attention"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -181,6 +186,37 @@ def sparse_attention(d: Dims, q, k_cache, v_cache, meta, page_table, seq_lens, p
         int(prefix), int(window), int(budget), float(scale), _ptr(sel, torch.int32, "sel"),
         _ptr(n_sel, torch.int32, "n_sel"), _ptr(out, bf, "out"), _ptr(lse, torch.float32, "lse"),
         _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def select_scores(d: Dims, scores, seq_lens, prefix: int, window: int, budget: int, sel, n_sel,
+                  ws, stream=None):
+    """Top-k pages over given fp32 scores [B][Hkv][max_pages_per_seq] (the
+    selection csa_score_select makes from its own scores)."""
+    _check("csa_select_scores", lib().csa_select_scores(
+        ctypes.byref(d), _ptr(scores, torch.float32, "scores"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), int(prefix), int(window), int(budget),
+        _ptr(sel, torch.int32, "sel"), _ptr(n_sel, torch.int32, "n_sel"), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def shard_selection(d: Dims, sel, n_sel, page_lo: int, page_hi: int, sel_local, n_sel_local,
+                    stream=None):
+    """The selected pages in [page_lo, page_hi), as pages of that shard."""
+    _check("csa_shard_selection", lib().csa_shard_selection(
+        ctypes.byref(d), _ptr(sel, torch.int32, "sel"), _ptr(n_sel, torch.int32, "n_sel"),
+        int(page_lo), int(page_hi), int(sel_local.shape[-1]),
+        _ptr(sel_local, torch.int32, "sel_local"), _ptr(n_sel_local, torch.int32, "n_sel_local"),
+        _stream(stream)))
+
+
+def merge_attention(out_parts, lse_parts, out, lse=None, stream=None):
+    """Log-sum-exp merge of partial attentions over disjoint token sets:
+    out_parts bf16 [R][B][Hq][D], lse_parts fp32 [R][B][Hq]."""
+    R, B, Hq, D = out_parts.shape
+    _check("csa_merge_attention", lib().csa_merge_attention(
+        int(R), int(B), int(Hq), int(D), _ptr(out_parts, torch.bfloat16, "out_parts"),
+        _ptr(lse_parts, torch.float32, "lse_parts"), _ptr(out, torch.bfloat16, "out"),
+        _ptr(lse, torch.float32, "lse"), _stream(stream)))
 
 
 def meta8_row_bytes(D: int) -> int:

@@ -496,6 +496,75 @@ int csa_sparse_attention_fp8(const csa_dims* d, const void* q, const void* k_cac
                                    lse, workspace, workspace_bytes, stream);
 }
 
+int csa_select_scores(const csa_dims* d, const float* scores, const int32_t* seq_lens,
+                      int prefix, int window, int budget_tokens, int32_t* sel_pages,
+                      int32_t* n_sel, void* workspace, size_t workspace_bytes, void* stream) {
+    Shape s;
+    int rc = check_dims(d, &s);
+    if (rc != CSA_OK) return rc;
+    CSA_REQUIRE(scores);
+    CSA_REQUIRE(seq_lens);
+    CSA_REQUIRE(sel_pages);
+    CSA_REQUIRE(n_sel);
+    if (prefix < 0 || window < 0 || budget_tokens < 0) return CSA_ERR_INVALID_ARG;
+    const int k_pages = budget_tokens / kPage;
+    if (k_pages > s.max_sel) return CSA_ERR_INVALID_ARG;
+    WsLayout w;
+    rc = check_ws(s, workspace, workspace_bytes, &w);
+    if (rc != CSA_OK) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    note_stream_call(stream, kCallOther);
+    // the selection rewrites its scores in place: it works on a copy
+    float* ws_scores = at<float>(workspace, w.scores);
+    const size_t bytes = sizeof(float) * (size_t)s.B * s.Hkv * s.MP;
+    if (cudaMemcpyAsync(ws_scores, scores, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return launch_status(cudaGetLastError());
+    SelectParams lp;
+    lp.scores_ws = ws_scores;
+    lp.seq_lens = seq_lens;
+    lp.prefix = prefix;
+    lp.window = window;
+    lp.k_pages = k_pages;
+    lp.sel = sel_pages;
+    lp.n_sel = n_sel;
+    lp.keyrange = at<uint2>(workspace, w.keyrange);   // zero: the full key range
+    lp.flags = at<uint32_t>(workspace, w.flags);
+    lp.smem_keys = 0;
+    lp.s = s;
+    return launch_status(launch_select(lp, st));
+}
+
+int csa_shard_selection(const csa_dims* d, const int32_t* sel_pages, const int32_t* n_sel,
+                        int page_lo, int page_hi, int max_sel_local, int32_t* sel_local,
+                        int32_t* n_sel_local, void* stream) {
+    Shape s;
+    int rc = check_dims(d, &s);
+    if (rc != CSA_OK) return rc;
+    CSA_REQUIRE(sel_pages);
+    CSA_REQUIRE(n_sel);
+    CSA_REQUIRE(sel_local);
+    CSA_REQUIRE(n_sel_local);
+    if (page_lo < 0 || page_hi < page_lo || max_sel_local < s.max_sel) return CSA_ERR_INVALID_ARG;
+    note_stream_call(stream, kCallOther);
+    return launch_status(launch_shard_selection(s, sel_pages, n_sel, page_lo, page_hi,
+                                                max_sel_local, sel_local, n_sel_local,
+                                                (cudaStream_t)stream));
+}
+
+int csa_merge_attention(int parts, int batch, int q_heads, int head_dim, const void* out_parts,
+                        const float* lse_parts, void* out, float* lse, void* stream) {
+    if (parts < 1 || parts > 64 || batch < 1 || q_heads < 1) return CSA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128 && head_dim != 256) return CSA_ERR_INVALID_ARG;
+    if ((long long)batch * q_heads > (1ll << 30)) return CSA_ERR_INVALID_ARG;
+    CSA_REQUIRE(out_parts);
+    CSA_REQUIRE(lse_parts);
+    CSA_REQUIRE(out);
+    CSA_OPTIONAL(lse);
+    note_stream_call(stream, kCallOther);
+    return launch_status(launch_merge(parts, batch * q_heads, head_dim, out_parts, lse_parts,
+                                      out, lse, (cudaStream_t)stream));
+}
+
 int csa_get_device_status(void* workspace, void* stream, int* flags_out) {
     if (!workspace || !aligned16(workspace)) return CSA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;

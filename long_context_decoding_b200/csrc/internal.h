@@ -121,6 +121,13 @@ void note_stream_call(const void* stream, CallKind kind);
 CallKind last_stream_call(const void* stream);
 
 // Grid sizes (shared by the workspace sizing and the launches).
+// ---------------------------------------------------------------- context parallelism
+cudaError_t launch_shard_selection(const Shape& s, const int32_t* sel, const int32_t* n_sel,
+                                   int lo, int hi, int max_local, int32_t* sel_local,
+                                   int32_t* n_local, cudaStream_t st);
+cudaError_t launch_merge(int parts, int bh_count, int D, const void* out_parts,
+                         const float* lse_parts, void* out, float* lse, cudaStream_t st);
+
 int device_sm_count();
 int decode_grid(const Shape& s);
 size_t decode_record_floats(const Shape& s);   // floats per split-K partial record
