@@ -487,26 +487,40 @@ def run_ours(args, dist: Dist, base: wl.Workload):
 
 
 def e2e(st: Stack, K: int, W: int, dist: Dist):
-    """Per step: H2D copy of the step's q/new_k/new_v (pinned host memory),
-    the 24 library calls, D2H copy of every layer's output; one CUDA graph
-    per step, K steps timed."""
+    """Per step: one H2D copy of the step's inputs (every layer's q, new_k
+    and new_v, packed in one pinned host buffer), the 24 library calls on
+    views of the device copy, and one D2H copy of every layer's output
+    (the layers write into one device buffer); one CUDA graph per step, K
+    steps timed."""
     nl = len(st.layers)
-    host_in, dev_in, host_out = [], [], []
+    shapes = [[t.shape for t in st.inputs[0][li]] for li in range(nl)]
+    sizes = [[t.numel() for t in st.inputs[0][li]] for li in range(nl)]
+    per_step = sum(sum(x) for x in sizes)
+    dev = st.dev
+    dev_in = torch.empty(per_step, dtype=torch.bfloat16, device=dev)
+    views, at = [], 0
+    for li in range(nl):
+        v = []
+        for shp, n in zip(shapes[li], sizes[li]):
+            v.append(dev_in[at:at + n].view(shp))
+            at += n
+        views.append(v)
+    host_in = []
     for s in range(K + W):
-        hi = [[t.cpu().pin_memory() for t in st.inputs[s][li]] for li in range(nl)]
-        di = [[torch.empty_like(t) for t in st.inputs[s][li]] for li in range(nl)]
-        ho = [torch.empty(st.layers[li].out.shape, dtype=torch.bfloat16).pin_memory()
-              for li in range(nl)]
-        host_in.append(hi), dev_in.append(di), host_out.append(ho)
+        h = torch.cat([t.reshape(-1).cpu() for li in range(nl) for t in st.inputs[s][li]])
+        host_in.append(h.pin_memory())
+    out_all = torch.empty((nl,) + tuple(st.layers[0].out.shape), dtype=torch.bfloat16, device=dev)
+    saved = [lay.out for lay in st.layers]
+    for li, lay in enumerate(st.layers):
+        lay.out = out_all[li]
+    host_out = [torch.empty(out_all.shape, dtype=torch.bfloat16).pin_memory()
+                for _ in range(K + W)]
 
     def step(s):
-        for li in range(nl):
-            for d_, h_ in zip(dev_in[s][li], host_in[s][li]):
-                d_.copy_(h_, non_blocking=True)
-        st.calls(s, q=[x[0] for x in dev_in[s]], nk=[x[1] for x in dev_in[s]],
-                 nv=[x[2] for x in dev_in[s]])
-        for li in range(nl):
-            host_out[s][li].copy_(st.layers[li].out, non_blocking=True)
+        dev_in.copy_(host_in[s], non_blocking=True)
+        st.calls(s, q=[v[0] for v in views], nk=[v[1] for v in views],
+                 nv=[v[2] for v in views])
+        host_out[s].copy_(out_all, non_blocking=True)
 
     graphs = [st.graph(lambda s=s: step(s)) for s in range(K + W)]
     for s in range(W):
@@ -514,12 +528,16 @@ def e2e(st: Stack, K: int, W: int, dist: Dist):
     torch.cuda.synchronize()
     dist.barrier()
     t = dist.max(time_graphs(graphs[W:W + K]))
-    h2d = sum(t_.numel() * t_.element_size() for li in range(nl) for t_ in host_in[0][li])
-    d2h = sum(t_.numel() * t_.element_size() for t_ in host_out[0])
+    del graphs
+    for lay, o in zip(st.layers, saved):
+        lay.out = o
+    h2d = host_in[0].numel() * host_in[0].element_size()
+    d2h = host_out[0].numel() * host_out[0].element_size()
     return {"value": dist.world * st.w.B * nl * K / t, "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
-            "path": "pinned host -> device copies, csa_meta_update / csa_sparse_attention "
-                    "per layer, device -> pinned host copy of out; one CUDA graph per step"}
+            "path": "one pinned host -> device copy of the step's inputs (all layers' q, new "
+                    "K, new V), csa_meta_update / csa_sparse_attention per layer, one device -> "
+                    "pinned host copy of all layers' outputs; one CUDA graph per step"}
 
 
 def fp8_step(st: Stack, K: int, W: int, sc_buf, s_last: int, peak: float, dist: Dist):
