@@ -340,7 +340,8 @@ int csa_get_device_status(void *workspace, void *stream, int *flags_out);
 /* Static string for a status code (host). */
 const char *csa_status_string(int status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 102 (1.01 added the fp8-metadata
+ * entry points, 1.02 the context-parallel ones). */
 int csa_version(void);
 
 #ifdef __cplusplus

@@ -139,7 +139,7 @@ using namespace csa;
 
 extern "C" {
 
-int csa_version(void) { return 100; }
+int csa_version(void) { return 102; }
 
 const char* csa_status_string(int st) {
     switch (st) {

@@ -35,7 +35,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert L.csa_version() == 100
+    assert L.csa_version() == 102   # 1.02: the fp8 and context-parallel entry points
     assert csa.status_string(0) == "ok"
     assert "workspace" in csa.status_string(-3)
     assert csa.status_string(-99) == "unknown status"
