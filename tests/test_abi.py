@@ -97,6 +97,35 @@ def test_host_validation_codes(L):
     assert L.csa_get_device_status(None, None, None) == -3
 
 
+def test_host_validation_codes_fp8_and_context_parallel(L):
+    d = dims()
+    W = (FAKE, ctypes.c_size_t(1 << 40), None)
+    # fp8 scoring without the fp8 copy; fp8 update with a bad n_new
+    assert L.csa_score_select_fp8(ctypes.byref(d), FAKE, None, FAKE, FAKE, 0, 0, 64, FAKE, FAKE,
+                                  None, *W) == -1
+    assert L.csa_meta_update_fp8(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+                                 0, *W) == -1
+    # selection over given scores: null scores, budget over max_sel, no workspace
+    def sel(scores=FAKE, budget=64, ws=W):
+        return L.csa_select_scores(ctypes.byref(d), scores, FAKE, 0, 0, budget, FAKE, FAKE, *ws)
+    assert sel(scores=None) == -1
+    assert sel(scores=MISALIGNED) == -1
+    assert sel(budget=16 * 513) == -1
+    assert sel(ws=(FAKE, ctypes.c_size_t(16), None)) == -3
+    # shard selection: an empty or inverted range is fine / rejected; max_sel_local too small
+    assert L.csa_shard_selection(ctypes.byref(d), FAKE, FAKE, 10, 5, 512, FAKE, FAKE, None) == -1
+    assert L.csa_shard_selection(ctypes.byref(d), FAKE, FAKE, 0, 10, 511, FAKE, FAKE, None) == -1
+    assert L.csa_shard_selection(ctypes.byref(d), FAKE, None, 0, 10, 512, FAKE, FAKE, None) == -1
+    # merge: parts, head_dim, pointers
+    def merge(parts=2, D=128, out=FAKE):
+        return L.csa_merge_attention(parts, 4, 32, D, FAKE, FAKE, out, None, None)
+    assert merge(parts=0) == -1
+    assert merge(parts=65) == -1
+    assert merge(D=96) == -1
+    assert merge(out=None) == -1
+    assert merge(out=MISALIGNED) == -1
+
+
 def test_binding_requires_cuda_tensors():
     import torch
     d = dims(B=1, Hq=4, Hkv=1, max_pages_per_seq=4, num_pages=4, max_sel=4)
