@@ -690,6 +690,7 @@ def run_sweep(args, dist: Dist):
             t = graph_time(lambda: lay.step(c.q, fused=True), args.steps, args.warmup, flush)
             by = cost.layer_bytes(w.seq_lens, w.Hq, w.Hkv, w.D, w.prefix, w.window, budget)
             points.append({"L": L, "budget": "all" if budget is None else budget,
+                           "path": cost.path_of(L, w.prefix, w.window, budget),
                            "sparse_us": 1e6 * t, "dense_us": 1e6 * t_dense,
                            "speedup": t_dense / t, "sparse_bytes": by["sparse"],
                            "dense_bytes": by["dense"], "sparse_gbs": by["sparse"] / t / 1e9})
@@ -720,6 +721,7 @@ def run_sweep(args, dist: Dist):
             "points": points,
             "cost_model": {"t0_us": 1e6 * t0, "bw_gbs": 1.0 / slope / 1e9,
                            "max_rel_err": worst, "form": "t = t0 + algorithmic bytes / bw"},
+            "cost_model_per_path": cost.fit_per_path(points),
             "sparse_faster_than_dense_for_all_L_ge_32k": beats,
             "all_budget_min_speedup_vs_dense": all_ratio}
     if dist.rank == 0:

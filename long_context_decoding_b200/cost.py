@@ -63,3 +63,46 @@ def layer_bytes(seq_lens: Iterable[int], Hq: int, Hkv: int, D: int, prefix: int,
         dense += Hkv * int(L) * 4 * D
     qo = 2 * B * Hq * D * 2
     return {"meta": meta, "kv": kv, "q_out": qo, "sparse": meta + kv + qo, "dense": dense + qo}
+
+
+def path_of(L: int, prefix: int, window: int, budget) -> str:
+    """Which kernels a csa_sparse_attention call runs for a sequence of L
+    tokens: the prefix/window decode alone (no page to select), the dense
+    decode (every candidate kept: budget "all" or k >= the candidates) or
+    the one-call path (scoring, fused selection + attention, combine)."""
+    if budget is None or budget == "all":
+        return "dense"
+    u = unit_bytes(int(L), 1, prefix, window, int(budget))
+    if u.k_pages == 0:
+        return "prefix_window"
+    return "dense" if u.k_pages >= u.candidates else "one_call"
+
+
+def fit_per_path(points) -> dict:
+    """t = t0[path] + bytes / bw: one bandwidth, one fixed cost per path,
+    fitted by least squares on the relative error (weights 1 / t^2, so that
+    the short calls count as much as the long ones).  points: dicts with
+    "path" (path_of), "sparse_bytes", "sparse_us"."""
+    groups = {}
+    for p in points:
+        groups.setdefault(p["path"], []).append(
+            (float(p["sparse_bytes"]), float(p["sparse_us"]) * 1e-6))
+    # within each path: weighted means; then the shared slope
+    stats = {}
+    num = den = 0.0
+    for k, g in groups.items():
+        w = [1.0 / (y * y) for _, y in g]
+        sw = sum(w)
+        mx = sum(wi * x for wi, (x, _) in zip(w, g)) / sw
+        my = sum(wi * y for wi, (_, y) in zip(w, g)) / sw
+        stats[k] = (mx, my)
+        num += sum(wi * (x - mx) * (y - my) for wi, (x, y) in zip(w, g))
+        den += sum(wi * (x - mx) ** 2 for wi, (x, _) in zip(w, g))
+    slope = num / den
+    t0 = {k: my - slope * mx for k, (mx, my) in stats.items()}
+    worst = max(abs(t0[p["path"]] + slope * float(p["sparse_bytes"])
+                    - float(p["sparse_us"]) * 1e-6) / (float(p["sparse_us"]) * 1e-6)
+                for p in points)
+    return {"bw_gbs": 1.0 / slope / 1e9, "t0_us": {k: 1e6 * v for k, v in t0.items()},
+            "max_rel_err": worst,
+            "form": "t = t0[path] + algorithmic bytes / bw (least squares on relative error)"}
