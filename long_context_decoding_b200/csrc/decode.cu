@@ -22,8 +22,9 @@
 //
 // Per CTA and phase: the page ids of its slice are resolved once into shared
 // memory; every warp then streams its own pages (round-robin over the slice)
-// with 16-byte cp.async copies into a private double buffer, laid out with
-// the 128-byte XOR swizzle (16-byte chunk c of token row r at c ^ (r & 7)),
+// with 16-byte cp.async copies into a private ring of K/V tile slots (four at
+// D <= 128, two at D = 256), laid out with the 128-byte XOR swizzle (16-byte
+// chunk c of token row r at c ^ (r & 7)),
 // so ldmatrix reads it without bank conflicts; slots past the end of the
 // sequence are zero-filled by the copy itself.  (Per-page TMA copies were
 // measured slower here: their issue cost, paid serially by one thread, caps
