@@ -43,8 +43,9 @@ template <int D, int NB>
 struct FusedCfg {
     static constexpr int kWarps = 8;                    // == kClThreads / 32
     // K/V tile slots per warp: two keep two CTAs per SM at D <= 128 (three
-    // slots, with smaller item lists, measured no faster)
-    static constexpr int kHalves = 2;
+    // slots, with smaller item lists, measured no faster); at D = 256 one CTA
+    // fills the SM either way and a third slot fits
+    static constexpr int kHalves = D == 256 ? 3 : 2;
     using Tile = TileCfg<D, NB, kWarps, kHalves>;
     static constexpr size_t kItems = (size_t)kFusedItems * 8;
     static constexpr size_t kUnits = (size_t)(kFusedUnits + 1) * 4 + (size_t)kFusedUnits * 4;
@@ -52,6 +53,10 @@ struct FusedCfg {
                                     kItems + kFusedItems * 4 /* share */ + kUnits;
 };
 static_assert(kClThreads == 256, "the fused kernel runs 8 warps per CTA");
+static_assert(FusedCfg<256, 2>::kSmem + sizeof(ClShared) + 1024 <= 232448,
+              "one fused CTA fits an SM at D = 256");
+static_assert(2 * (FusedCfg<128, 1>::kSmem + sizeof(ClShared) + 1024) <= 233472,
+              "two fused CTAs fit an SM at D <= 128");
 
 template <int D, int NB>
 __global__ void __cluster_dims__(kCl, 1, 1)

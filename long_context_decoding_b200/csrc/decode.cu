@@ -51,7 +51,7 @@ struct DecCfg {
     // so that three fit beside a CTA of the selection kernel when both are
     // resident (16 heads would spill at that bound)
     static constexpr int kMinBlocks = D == 256 ? 1 : (NB == 1 ? 4 : 3);
-    static constexpr int kHalves = D == 256 ? 2 : 4;    // K/V tile slots per warp
+    static constexpr int kHalves = D == 256 ? 3 : 4;    // K/V tile slots per warp
     using Tile = TileCfg<D, NB, kWarps, kHalves>;
     static constexpr size_t kStageArea = Tile::kStageArea;
     static constexpr size_t kMl = Tile::kMl;
