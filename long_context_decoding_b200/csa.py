@@ -121,6 +121,28 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _sizes(d: Dims, n_new: int = 1) -> dict:
+    """Elements each named argument of dims d must hold, at least (the C
+    calls index them by d's sizes)."""
+    B, Hq, Hkv, D = d.B, d.Hq, d.Hkv, d.D
+    NPG, MP = d.num_pages, d.max_pages_per_seq
+    return {"q": B * Hq * D, "out": B * Hq * D, "lse": B * Hq,
+            "k_cache": NPG * Hkv * 16 * D, "v_cache": NPG * Hkv * 16 * D,
+            "meta": NPG * Hkv * 2 * D, "meta8": NPG * Hkv * (2 * D + 16),
+            "page_table": B * MP, "seq_lens": B, "sel": B * Hkv * d.max_sel, "n_sel": B * Hkv,
+            "scores": B * Hkv * MP, "scores_out": B * Hkv * MP,
+            "new_k": B * n_new * Hkv * D, "new_v": B * n_new * Hkv * D}
+
+
+def _check_sizes(d: Dims, n_new: int = 1, **tensors):
+    """Raise ValueError when a tensor is smaller than dims d require: a call
+    would read or write past its end."""
+    need = _sizes(d, max(1, int(n_new)))
+    for name, t in tensors.items():
+        if t is not None and t.numel() < need[name]:
+            raise ValueError(f"{name} holds {t.numel()} elements; dims need {need[name]}")
+
+
 def workspace_size(d: Dims) -> int:
     n = lib().csa_workspace_size(ctypes.byref(d))
     if n == 0:
@@ -139,6 +161,8 @@ def new_workspace(d: Dims, device="cuda", stream=None) -> torch.Tensor:
 def meta_update(d: Dims, k_cache, v_cache, meta, page_table, seq_lens, new_k, new_v, n_new: int,
                 ws, stream=None):
     """Append n_new tokens per sequence (new_k/new_v None: rebuild metadata)."""
+    _check_sizes(d, n_new, k_cache=k_cache, v_cache=v_cache, meta=meta, page_table=page_table,
+                 seq_lens=seq_lens, new_k=new_k, new_v=new_v)
     bf = torch.bfloat16
     _check("csa_meta_update", lib().csa_meta_update(
         ctypes.byref(d), _ptr(k_cache, bf, "k_cache"), _ptr(v_cache, bf, "v_cache"),
@@ -150,6 +174,8 @@ def meta_update(d: Dims, k_cache, v_cache, meta, page_table, seq_lens, new_k, ne
 def score_select(d: Dims, q, meta, page_table, seq_lens, prefix: int, window: int, budget: int,
                  sel, n_sel, ws, scores_out=None, stream=None):
     """Quest scores from metadata and top-k page selection into sel / n_sel."""
+    _check_sizes(d, q=q, meta=meta, page_table=page_table, seq_lens=seq_lens, sel=sel,
+                 n_sel=n_sel, scores_out=scores_out)
     bf = torch.bfloat16
     _check("csa_score_select", lib().csa_score_select(
         ctypes.byref(d), _ptr(q, bf, "q"), _ptr(meta, bf, "meta"),
@@ -162,6 +188,8 @@ def score_select(d: Dims, q, meta, page_table, seq_lens, prefix: int, window: in
 def decode(d: Dims, q, k_cache, v_cache, page_table, seq_lens, sel, n_sel, prefix: int,
            window: int, out, ws, lse=None, scale: float = 0.0, stream=None):
     """Combined sparse attention over prefix + window + selected pages."""
+    _check_sizes(d, q=q, k_cache=k_cache, v_cache=v_cache, page_table=page_table,
+                 seq_lens=seq_lens, sel=sel, n_sel=n_sel, out=out, lse=lse)
     bf = torch.bfloat16
     _check("csa_decode", lib().csa_decode(
         ctypes.byref(d), _ptr(q, bf, "q"), _ptr(k_cache, bf, "k_cache"),
@@ -178,6 +206,8 @@ def sparse_attention(d: Dims, q, k_cache, v_cache, meta, page_table, seq_lens, p
     """Scoring, top-k selection and the sparse decode in one call (the
     selection and the decode of the selected pages share a launch when the
     shape allows)."""
+    _check_sizes(d, q=q, k_cache=k_cache, v_cache=v_cache, meta=meta, page_table=page_table,
+                 seq_lens=seq_lens, sel=sel, n_sel=n_sel, out=out, lse=lse)
     bf = torch.bfloat16
     _check("csa_sparse_attention", lib().csa_sparse_attention(
         ctypes.byref(d), _ptr(q, bf, "q"), _ptr(k_cache, bf, "k_cache"),
@@ -192,6 +222,7 @@ def select_scores(d: Dims, scores, seq_lens, prefix: int, window: int, budget: i
                   ws, stream=None):
     """Top-k pages over given fp32 scores [B][Hkv][max_pages_per_seq] (the
     selection csa_score_select makes from its own scores)."""
+    _check_sizes(d, scores=scores, seq_lens=seq_lens, sel=sel, n_sel=n_sel)
     _check("csa_select_scores", lib().csa_select_scores(
         ctypes.byref(d), _ptr(scores, torch.float32, "scores"),
         _ptr(seq_lens, torch.int32, "seq_lens"), int(prefix), int(window), int(budget),
@@ -202,6 +233,9 @@ def select_scores(d: Dims, scores, seq_lens, prefix: int, window: int, budget: i
 def shard_selection(d: Dims, sel, n_sel, page_lo: int, page_hi: int, sel_local, n_sel_local,
                     stream=None):
     """The selected pages in [page_lo, page_hi), as pages of that shard."""
+    _check_sizes(d, sel=sel, n_sel=n_sel)
+    if sel_local.numel() < d.B * d.Hkv * sel_local.shape[-1] or n_sel_local.numel() < d.B * d.Hkv:
+        raise ValueError("sel_local / n_sel_local smaller than [B][Hkv][...]")
     _check("csa_shard_selection", lib().csa_shard_selection(
         ctypes.byref(d), _ptr(sel, torch.int32, "sel"), _ptr(n_sel, torch.int32, "n_sel"),
         int(page_lo), int(page_hi), int(sel_local.shape[-1]),
@@ -213,6 +247,9 @@ def merge_attention(out_parts, lse_parts, out, lse=None, stream=None):
     """Log-sum-exp merge of partial attentions over disjoint token sets:
     out_parts bf16 [R][B][Hq][D], lse_parts fp32 [R][B][Hq]."""
     R, B, Hq, D = out_parts.shape
+    if lse_parts.numel() < R * B * Hq or out.numel() < B * Hq * D or \
+            (lse is not None and lse.numel() < B * Hq):
+        raise ValueError("lse_parts [R][B][Hq], out [B][Hq][D] and lse [B][Hq] must match out_parts")
     _check("csa_merge_attention", lib().csa_merge_attention(
         int(R), int(B), int(Hq), int(D), _ptr(out_parts, torch.bfloat16, "out_parts"),
         _ptr(lse_parts, torch.float32, "lse_parts"), _ptr(out, torch.bfloat16, "out"),
@@ -233,6 +270,8 @@ def new_meta8(d: Dims, device="cuda") -> torch.Tensor:
 def meta_update_fp8(d: Dims, k_cache, v_cache, meta, meta8, page_table, seq_lens, new_k, new_v,
                     n_new: int, ws, stream=None):
     """csa_meta_update that also keeps the fp8 copy meta8 current."""
+    _check_sizes(d, n_new, k_cache=k_cache, v_cache=v_cache, meta=meta, meta8=meta8,
+                 page_table=page_table, seq_lens=seq_lens, new_k=new_k, new_v=new_v)
     bf = torch.bfloat16
     _check("csa_meta_update_fp8", lib().csa_meta_update_fp8(
         ctypes.byref(d), _ptr(k_cache, bf, "k_cache"), _ptr(v_cache, bf, "v_cache"),
@@ -245,6 +284,8 @@ def meta_update_fp8(d: Dims, k_cache, v_cache, meta, meta8, page_table, seq_lens
 def score_select_fp8(d: Dims, q, meta8, page_table, seq_lens, prefix: int, window: int,
                      budget: int, sel, n_sel, ws, scores_out=None, stream=None):
     """csa_score_select with the scores from the fp8 metadata copy."""
+    _check_sizes(d, q=q, meta8=meta8, page_table=page_table, seq_lens=seq_lens, sel=sel,
+                 n_sel=n_sel, scores_out=scores_out)
     _check("csa_score_select_fp8", lib().csa_score_select_fp8(
         ctypes.byref(d), _ptr(q, torch.bfloat16, "q"), _ptr(meta8, torch.uint8, "meta8"),
         _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
@@ -257,6 +298,8 @@ def sparse_attention_fp8(d: Dims, q, k_cache, v_cache, meta8, page_table, seq_le
                          prefix: int, window: int, budget: int, sel, n_sel, out, ws, lse=None,
                          scale: float = 0.0, stream=None):
     """csa_sparse_attention with the scores from the fp8 metadata copy."""
+    _check_sizes(d, q=q, k_cache=k_cache, v_cache=v_cache, meta8=meta8, page_table=page_table,
+                 seq_lens=seq_lens, sel=sel, n_sel=n_sel, out=out, lse=lse)
     bf = torch.bfloat16
     _check("csa_sparse_attention_fp8", lib().csa_sparse_attention_fp8(
         ctypes.byref(d), _ptr(q, bf, "q"), _ptr(k_cache, bf, "k_cache"),
@@ -270,6 +313,8 @@ def sparse_attention_fp8(d: Dims, q, k_cache, v_cache, meta8, page_table, seq_le
 def decode_full(d: Dims, q, k_cache, v_cache, page_table, seq_lens, out, ws, lse=None,
                 scale: float = 0.0, stream=None):
     """Dense decode over every valid token (the unmodified layer)."""
+    _check_sizes(d, q=q, k_cache=k_cache, v_cache=v_cache, page_table=page_table,
+                 seq_lens=seq_lens, out=out, lse=lse)
     bf = torch.bfloat16
     _check("csa_decode_full", lib().csa_decode_full(
         ctypes.byref(d), _ptr(q, bf, "q"), _ptr(k_cache, bf, "k_cache"),
@@ -286,6 +331,8 @@ def decode_noalloc(d: Dims, q, k_cache, v_cache, page_table, seq_lens, sel, n_se
     inside the library, shared by every call on the device, so calls must
     not overlap on the GPU.  Device-side flags of this call are not
     reported."""
+    _check_sizes(d, q=q, k_cache=k_cache, v_cache=v_cache, page_table=page_table,
+                 seq_lens=seq_lens, sel=sel, n_sel=n_sel, out=out, lse=lse)
     f = lib().csa_decode_noalloc
     P = ctypes.c_void_p
     f.argtypes = [ctypes.POINTER(Dims), P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,

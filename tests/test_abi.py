@@ -126,6 +126,23 @@ def test_host_validation_codes_fp8_and_context_parallel(L):
     assert merge(out=MISALIGNED) == -1
 
 
+def test_binding_checks_tensor_sizes():
+    """A tensor smaller than the dims say is rejected before any call (the
+    kernels would run past its end)."""
+    import torch
+    d = dims(B=2, Hq=8, Hkv=2, D=64, max_pages_per_seq=10, num_pages=30, max_sel=4)
+    csa._check_sizes(d, q=torch.empty(2 * 8 * 64), k_cache=torch.empty(30 * 2 * 16 * 64),
+                     sel=torch.empty(2, 2, 4), n_sel=torch.empty(2, 2))
+    for kw in (dict(q=torch.empty(2, 8, 63)), dict(k_cache=torch.empty(29, 2, 16, 64)),
+               dict(meta=torch.empty(30, 2, 2, 32)), dict(page_table=torch.empty(2, 9)),
+               dict(sel=torch.empty(2, 2, 3)), dict(lse=torch.empty(2, 7)),
+               dict(scores_out=torch.empty(2, 2, 9)), dict(meta8=torch.empty(30, 2, 143))):
+        with pytest.raises(ValueError):
+            csa._check_sizes(d, **kw)
+    with pytest.raises(ValueError):                  # three new tokens need 3x the rows
+        csa._check_sizes(d, 3, new_k=torch.empty(2, 2, 2, 64))
+
+
 def test_binding_requires_cuda_tensors():
     import torch
     d = dims(B=1, Hq=4, Hkv=1, max_pages_per_seq=4, num_pages=4, max_sel=4)
