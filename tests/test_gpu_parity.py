@@ -337,6 +337,39 @@ def test_one_call_many_units_uses_separate_kernels(cuda):
     check_one_call(Run(wl.make_case(w, cuda)), oracle_too=False)
 
 
+@pytest.mark.parametrize("window", [0, 15, 16, 64])
+def test_one_call_right_after_append(window, cuda):
+    """The one-call step issued straight after a one-token append, with the
+    appended page inside the window (16 tokens or more) or a candidate
+    (fewer): the step equals the same step on metadata rebuilt afterwards,
+    bit for bit, and the oracle."""
+    w = small(B=2, Hq=8, Hkv=2, D=128, lens=(1000, 1517), prefix=16, window=window,
+              budget=128, extra=3)
+    case = wl.make_case(w, cuda)
+    run = Run(case)
+    run.gpu_meta()
+    for s in range(3):
+        nk, nv = wl.step_tokens(case, s)[1:]
+        case.seq_lens += 1
+        csa.meta_update(run.d, case.k_cache, case.v_cache, run.layer.meta, case.page_table,
+                        case.seq_lens, nk, nv, 1, run.ws)
+        sel_a, nsel_a, out_a, lse_a = sparse_call(run)
+    torch.cuda.synchronize()
+    assert csa.device_status(run.ws) == 0
+    meta_after = run.layer.meta.clone()
+    run.refresh_host()
+    run.gpu_meta()
+    assert torch.equal(run.layer.meta, meta_after)
+    sel_b, nsel_b, out_b, lse_b = sparse_call(run)
+    torch.cuda.synchronize()
+    assert torch.equal(nsel_a, nsel_b) and torch.equal(sel_a, sel_b)
+    assert torch.equal(out_a, out_b)
+    assert torch.equal(torch.isfinite(lse_a), torch.isfinite(lse_b))
+    fin = torch.isfinite(lse_b)
+    assert torch.equal(lse_a[fin], lse_b[fin])
+    check_one_call(run)
+
+
 def test_one_call_repeated_and_after_appends(cuda):
     """Back-to-back one-call steps with appends in between, no host syncs."""
     w = replace(wl.CTX32K, steps=4)
