@@ -166,7 +166,6 @@ __global__ void __cluster_dims__(kCl, 1, 1)
     const int c_lo = sg.c_lo;
     const int lo = kk * rank / kCl, hi = kk * (rank + 1) / kCl;   // this CTA's share
     int32_t* out = P.sel + (size_t)u * p.s.max_sel;
-    cluster_select_begin(sh);
     if (tid < G * D / 64) {     // this unit's queries (a caller input) into L1
         const uint16_t* qrow = p.q + ((size_t)b * p.s.Hq + (size_t)(u % Hkv) * G) * D + tid * 64;
         asm volatile("prefetch.global.L1 [%0];" ::"l"(qrow));
@@ -189,7 +188,7 @@ __global__ void __cluster_dims__(kCl, 1, 1)
                            int* d = cl.map_shared_rank(share, dst);
                            d[pos - kk * dst / kCl] = c_lo + i;
                        });
-        cl.sync();              // every share is complete
+        cluster_sync_all();     // every share is complete; no remote access after this
     }
     if (rank == 0 && tid == 0) {   // every CTA read the key range before the last barrier
         P.n_sel[u] = kk;

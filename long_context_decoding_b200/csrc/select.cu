@@ -304,7 +304,6 @@ select_cluster_kernel(SelectParams p) {
     const int n = sg.c_hi - sg.c_lo;
     const int kk = p.k_pages < n ? p.k_pages : n;
     int32_t* out = p.sel + (size_t)u * p.s.max_sel;
-    cluster_select_begin(sh);
     pdl_wait();                 // scores and the previous readers of sel
     pdl_launch_dependents();
 
@@ -329,6 +328,7 @@ select_cluster_kernel(SelectParams p) {
     key_range(p.keyrange[u], kmin, kmax);
     cluster_select(cl, sh, p.scores_ws + (size_t)u * MP + c_lo, n, kk, kmin, kmax,
                    [&](int pos, int i) { out[pos] = c_lo + i; });
+    cluster_sync_all();         // no CTA's shared memory is read after this
     if (rank == 0 && tid == 0) {   // every CTA read the range before the last barrier
         p.n_sel[u] = kk;
         p.keyrange[u] = make_uint2(0u, 0u);

@@ -8,14 +8,17 @@
 // top-k); ties go to the lower logical page.  The 8 CTAs of a cluster (256
 // threads, 8 keys per thread in registers, up to 16384 candidates) turn the
 // fp32 scores into order-preserving uint32 keys, strip the high bits every
-// key shares (cluster min/max), and run an MSB-first radix select with 8-bit
-// digits: local histograms are merged in rank 0's shared memory through
-// distributed shared memory, every CTA reads the merged histogram and finds
-// the same digit, and a pass ends the search early when the bin holding the
-// k-th key is taken whole.  Per-warp, per-CTA and per-cluster prefixes of the
-// (above, equal) counts then give every selected candidate its position in
-// ascending index order: all keys above the threshold plus the lowest-index
-// keys equal to it.
+// key shares (the unit's key range from the scoring kernel), and run an
+// MSB-first radix select with 8-bit digits.  In each pass every CTA builds
+// its histogram in its own shared memory, one cluster barrier publishes
+// them, and every CTA reads all 8 through distributed shared memory (one
+// round trip), sums them and finds the same digit; a pass ends the search
+// early when the bin holding the k-th key is taken whole.  The same reads
+// give every CTA each rank's count of keys above the digit and in it, so
+// after the last pass every CTA knows each rank's (above, equal) totals
+// without another exchange, and per-warp prefixes give every selected
+// candidate its position in ascending index order: all keys above the
+// threshold plus the lowest-index keys equal to it.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -47,30 +50,19 @@ constexpr int kClCap = kCl * kClThreads * kClKeys;  // 16384 candidates
 constexpr int kClPasses = 4;                        // at most four 8-bit digits
 
 struct ClShared {
-    uint32_t hist[kClPasses][256];   // rank 0: merged histogram of each pass
-    uint32_t local[256];             // this CTA's histogram
-    uint32_t cgt[kCl], ceq[kCl];     // every CTA: the (above, equal) counts of each rank
+    uint32_t hist[2][256];           // this CTA's histogram, by pass parity
+    uint32_t rgt[kClWarps][kCl];     // per warp: each rank's keys above the digit
+    uint32_t req[kCl];               // each rank's keys in the digit's bin
+    uint32_t cgt[kCl], ceq[kCl];     // each rank's (above, equal) totals
     uint32_t red[kClWarps], wgt[kClWarps], weq[kClWarps];
     uint32_t digit, gt, cnt;
 };
 
-// Split cluster barrier (arrive now, wait later) with release / acquire
-// semantics on the cluster's shared memory.
-__device__ __forceinline__ void cluster_arrive() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Empties rank 0's merge buffers and arrives at the cluster barrier that
-// publishes them; call before the dependency wait (it touches only this
-// CTA's shared memory).  cluster_select waits on that barrier before its
-// first remote access.
-__device__ __forceinline__ void cluster_select_begin(ClShared& sh) {
-    for (int i = threadIdx.x; i < kClPasses * 256; i += kClThreads) (&sh.hist[0][0])[i] = 0;
-    __syncthreads();
-    cluster_arrive();
+// Cluster barrier with release / acquire semantics on the cluster's shared
+// memory (every thread of every CTA).
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Key range of a unit as published by the scoring kernel: x = ~min key,
@@ -86,17 +78,18 @@ __device__ __forceinline__ void key_range(uint2 r, uint32_t& kmin, uint32_t& kma
 }
 
 // Selects the kk largest of the n scores sc[0, n) (0 < kk < n <= kClCap),
-// whose order keys all lie in [kmin, kmax], with the CTAs of the cluster;
-// calls emit(pos, i) for every selected candidate i in this CTA's share, pos
-// being its rank in ascending index order.  Called by every thread of all
-// kCl CTAs after cluster_select_begin; ends with a cluster barrier, after
-// which no CTA reads another's shared memory.
+// whose order keys all lie in [kmin, kmax] (a key outside is clamped into
+// it, so a stale range still gives kk distinct positions), with the CTAs of
+// the cluster; calls emit(pos, i) for every selected candidate i in this
+// CTA's share, pos being its rank in ascending index order.  Called by every
+// thread of all kCl CTAs.  The last remote access is a read before emit; the
+// caller ends with a cluster barrier (cluster_sync_all) after emit and
+// before any CTA exits.
 template <typename Emit>
 __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float* sc, int n, int kk,
                                uint32_t kmin, uint32_t kmax, Emit emit) {
     const int rank = (int)cl.block_rank();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    ClShared* sh0 = cl.map_shared_rank(&sh, 0);
 
     // this CTA's chunk of the candidates; warp w holds a span, lane l the
     // keys span_lo + 32 j + l (coalesced loads)
@@ -109,16 +102,21 @@ __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float*
 #pragma unroll
     for (int j = 0; j < kClKeys; ++j) {
         const int i = wlo + 32 * j + lane;
-        kr[j] = order_key(__ldcg(sc + (i < whi ? i : 0)));
+        const uint32_t k = order_key(__ldcg(sc + (i < whi ? i : 0)));
+        kr[j] = k < kmin ? kmin : (k > kmax ? kmax : k);
     }
-    cluster_wait();             // rank 0's buffers are empty everywhere
 
     uint32_t pmask, pval;
     uint32_t remaining = (uint32_t)kk;
     bool take_all = false;
+    uint32_t gt_acc = 0;        // thread r < kCl: rank r's keys above the digits so far
     if (kmin == kmax) {
         pmask = 0xffffffffu;
         pval = kmax;
+        if (tid < kCl) {        // every key equal: a rank's count is its chunk's size
+            const int lo = tid * chunk, hi = lo + chunk < n ? lo + chunk : n;
+            sh.req[tid] = hi > lo ? (uint32_t)(hi - lo) : 0u;
+        }
     } else {
         int hb = 31 - __clz(kmin ^ kmax);
         pmask = hb >= 31 ? 0u : (0xffffffffu << (hb + 1));
@@ -126,17 +124,23 @@ __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float*
         for (int pass = 0;; ++pass) {
             const int lo_bit = hb - 7 > 0 ? hb - 7 : 0;
             const uint32_t dmask = (1u << (hb - lo_bit + 1)) - 1u;
-            sh.local[tid] = 0;
+            // the buffer of this parity was last read by the other CTAs in
+            // pass - 2, before they arrived at the barrier of pass - 1
+            uint32_t* hl = sh.hist[pass & 1];
+            hl[tid] = 0;
             __syncthreads();
 #pragma unroll
             for (int j = 0; j < kClKeys; ++j)
                 if (wlo + 32 * j + lane < whi && (kr[j] & pmask) == pval)
-                    atomicAdd(&sh.local[(kr[j] >> lo_bit) & dmask], 1u);
-            __syncthreads();
-            if (sh.local[tid]) atomicAdd(&sh0->hist[pass][tid], sh.local[tid]);
-            cl.sync();
-            // every CTA reads the merged histogram and finds the same digit
-            const uint32_t vbin = sh0->hist[pass][255 - tid];   // descending digit order
+                    atomicAdd(&hl[(kr[j] >> lo_bit) & dmask], 1u);
+            cluster_sync_all();             // every CTA's histogram is complete
+            // bin 255 - tid of every rank (descending digit order)
+            uint32_t h[kCl];
+#pragma unroll
+            for (int r = 0; r < kCl; ++r) h[r] = cl.map_shared_rank(hl, r)[255 - tid];
+            uint32_t vbin = 0;
+#pragma unroll
+            for (int r = 0; r < kCl; ++r) vbin += h[r];
             uint32_t incl = vbin;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -151,9 +155,24 @@ __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float*
                 sh.digit = 255 - tid;
                 sh.gt = gtc;
                 sh.cnt = vbin;
+#pragma unroll
+                for (int r = 0; r < kCl; ++r) sh.req[r] = h[r];
             }
             __syncthreads();
             const uint32_t d = sh.digit, gt = sh.gt, cnt = sh.cnt;
+            // each rank's keys in the bins above the digit (this thread's bin
+            // is 255 - tid)
+            const bool above = (uint32_t)(255 - tid) > d;
+#pragma unroll
+            for (int r = 0; r < kCl; ++r) {
+                const uint32_t v = __reduce_add_sync(0xffffffffu, above ? h[r] : 0u);
+                if (lane == 0) sh.rgt[warp][r] = v;
+            }
+            __syncthreads();
+            if (tid < kCl) {
+#pragma unroll
+                for (int w = 0; w < kClWarps; ++w) gt_acc += sh.rgt[w][tid];
+            }
             remaining -= gt;
             pval |= d << lo_bit;
             pmask |= dmask << lo_bit;
@@ -166,9 +185,13 @@ __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float*
         }
     }
     const uint32_t eq_take = take_all ? 0xffffffffu : remaining;
+    if (tid < kCl) {
+        sh.cgt[tid] = gt_acc;
+        sh.ceq[tid] = sh.req[tid];
+    }
 
-    // compaction: per-warp, per-CTA and per-cluster prefixes of (above, equal);
-    // every CTA sends its totals to every CTA, so one barrier suffices
+    // compaction: per-warp prefixes of (above, equal) in this CTA, on top of
+    // the lower ranks' totals
     uint32_t cgt = 0, ceq = 0;
 #pragma unroll
     for (int j = 0; j < kClKeys; ++j) {
@@ -184,12 +207,6 @@ __device__ void cluster_select(cg::cluster_group& cl, ClShared& sh, const float*
     __syncthreads();
     uint32_t gt_base = warp_prefix(sh.wgt, kClWarps);
     uint32_t eq_base = warp_prefix(sh.weq, kClWarps);
-    if (tid >= kClThreads - kCl) {   // last warp (its gt_base + cgt is the CTA's total)
-        ClShared* dst = cl.map_shared_rank(&sh, tid - (kClThreads - kCl));
-        dst->cgt[rank] = gt_base + cgt;
-        dst->ceq[rank] = eq_base + ceq;
-    }
-    cl.sync();                  // counts everywhere; no remote reads after this
     {
         const uint32_t x = lane < kCl && lane < rank ? sh.cgt[lane] : 0u;
         const uint32_t y = lane < kCl && lane < rank ? sh.ceq[lane] : 0u;
