@@ -94,7 +94,11 @@ __global__ void __cluster_dims__(kCl, 1, 1)
 
     if ((int)blockIdx.x >= n_sel_ctas) {
         // ------------------------------------------- prefix/window role
-        const int c0 = (int)blockIdx.x - n_sel_ctas, n0 = (int)gridDim.x - n_sel_ctas;
+        // work slot of this CTA: rank-major over the role's clusters (n0 is
+        // a multiple of 8), so that the slots in use, the first n_cta, fall
+        // in as many clusters, and so SMs, as there are slots
+        const int n0 = (int)gridDim.x - n_sel_ctas, rel = (int)blockIdx.x - n_sel_ctas;
+        const int c0 = (rel % kCl) * (n0 / kCl) + rel / kCl;
         for (int u = tid; u < units; u += kClThreads) {
             int L = p.seq_lens[u / Hkv];
             if (L < 0 || L > MP * kPage) L = 0;          // flagged by the scoring kernel
@@ -232,6 +236,64 @@ cudaError_t launch_fused_t(const FusedParams& p, cudaStream_t st) {
     return launch_combine(p.d, st);
 }
 
+// Clusters of the fused kernel that are resident at once on the current
+// device (clusters of 8 must sit in one GPC, so this is below SMs x CTAs per
+// SM / 8); 0 when the query fails.
+template <int D, int NB>
+int resident_clusters_t() {
+    static int cache[64] = {0};   // per device: the count, or -1 after a failed query
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && cache[dev] != 0) return cache[dev] > 0 ? cache[dev] : 0;
+    using C = FusedCfg<D, NB>;
+    auto kern = fused_kernel<D, NB>;
+    int n = 0;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmem);
+    if (e == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kCl * 64);
+        cfg.blockDim = dim3(kClThreads);
+        cfg.dynamicSmemBytes = C::kSmem;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    if (dev < 64) cache[dev] = n > 0 ? n : -1;
+    return n > 0 ? n : 0;
+}
+
+int resident_clusters(const Shape& s) {
+    const int nb = s.G > 8 ? 2 : 1;
+    switch (s.D * 10 + nb) {
+        case 641: return resident_clusters_t<64, 1>();
+        case 642: return resident_clusters_t<64, 2>();
+        case 1281: return resident_clusters_t<128, 1>();
+        case 1282: return resident_clusters_t<128, 2>();
+        case 2561: return resident_clusters_t<256, 1>();
+        case 2562: return resident_clusters_t<256, 2>();
+        default: return 0;
+    }
+}
+
+// Least CTAs of the prefix/window role for a call: no slice may exceed the
+// item capacity (every unit's fixed list holds at most ceil(prefix / 16) +
+// ceil(window / 16) + 2 pages).
+long long phase0_min_ctas(const Shape& s, long long prefix, long long window) {
+    const long long units = (long long)s.B * s.Hkv;
+    long long fixed = (prefix + kPage - 1) / kPage + (window + kPage - 1) / kPage + 2;
+    if (fixed > (long long)s.MP + 2) fixed = (long long)s.MP + 2;
+    return (units * fixed + kFusedItems - 1) / kFusedItems;
+}
+
+long long round_to_clusters(long long n0) {
+    if (n0 < kCl) n0 = kCl;
+    n0 = (n0 + kCl - 1) / kCl * kCl;
+    return n0 < (1ll << 30) ? n0 : (1ll << 30);
+}
+
 }  // namespace
 
 // The fused path serves up to 32 units, with at most kClCap candidates per
@@ -241,28 +303,35 @@ bool fused_eligible(const Shape& s, int prefix, int window, int k_pages) {
     return k_pages > 0 && (long long)s.B * s.Hkv <= kFusedUnits && n_max <= kClCap;
 }
 
-// CTAs of the prefix/window role for a call: what stays of the resident
-// capacity beside the selection clusters, at least enough that no slice
-// exceeds the item capacity (every unit's fixed list holds at most
-// ceil(prefix / 16) + ceil(window / 16) + 2 pages), and a whole number of
-// clusters.
-int fused_phase0_ctas(const Shape& s, long long prefix, long long window) {
+// The most CTAs of the prefix/window role any call of the shape launches
+// (for the workspace): what stays of two (or one) CTAs per SM beside the
+// selection clusters, at least the item capacity's minimum, whole clusters.
+int fused_phase0_ctas(const Shape& s) {
     const long long units = (long long)s.B * s.Hkv;
     const int per_sm = (s.D <= 128 && s.G <= 8) ? 2 : 1;
+    const long long all = (long long)s.MP * kPage;
     long long n0 = (long long)per_sm * device_sm_count() - kCl * units;
-    long long fixed = (prefix + kPage - 1) / kPage + (window + kPage - 1) / kPage + 2;
-    if (fixed > (long long)s.MP + 2) fixed = (long long)s.MP + 2;
-    const long long cap = (units * fixed + kFusedItems - 1) / kFusedItems;
-    if (n0 < cap) n0 = cap;
-    if (n0 < kCl) n0 = kCl;
-    n0 = (n0 + kCl - 1) / kCl * kCl;
-    return (int)(n0 < (1ll << 30) ? n0 : (1ll << 30));
+    const long long need = phase0_min_ctas(s, all, all);
+    return (int)round_to_clusters(n0 > need ? n0 : need);
 }
 
-// The most any call of the shape needs (for the workspace).
-int fused_phase0_ctas(const Shape& s) {
-    const long long all = (long long)s.MP * kPage;
-    return fused_phase0_ctas(s, all, all);
+// CTAs of the prefix/window role for a call: the clusters that stay resident
+// beside the selection clusters (so that none of the role waits for a second
+// wave), at least the call's item-capacity minimum, at most the workspace's
+// count.
+int fused_phase0_ctas(const Shape& s, long long prefix, long long window) {
+    const long long units = (long long)s.B * s.Hkv;
+    const long long most = fused_phase0_ctas(s);
+    long long n0 = most;
+    const int resident = resident_clusters(s);
+    if (resident > units) {
+        const long long fit = ((long long)resident - units) * kCl;
+        if (fit < n0) n0 = fit;
+    }
+    const long long need = phase0_min_ctas(s, prefix, window);
+    if (n0 < need) n0 = need;
+    n0 = round_to_clusters(n0);
+    return (int)(n0 < most ? n0 : most);
 }
 
 cudaError_t launch_fused(const FusedParams& p, cudaStream_t st) {

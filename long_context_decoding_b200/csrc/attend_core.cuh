@@ -185,10 +185,15 @@ __device__ void attend_unit(const AttendArgs& A, int u, int L, const int2* items
     // ---- S^T = K Q^T for the page in the buffer at kbase, the mask and the
     // online softmax (exp2 domain); leaves P^T as B fragments in pb
     auto qk_softmax = [&](uint32_t kbase, int page, int mask, uint32_t (&pb)[NB][2]) {
-        float sacc[NB][4];
+        // two accumulator chains (even and odd k steps) at D <= 128, summed at
+        // the end (at D = 256 the second chain's registers cost more than the
+        // shorter chain saves)
+        constexpr bool kTwo = D <= 128;
+        float sacc[NB][4], sacc2[NB][4];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
-            sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sacc[nb][i] = sacc2[nb][i] = 0.f;
 #pragma unroll
         for (int kb = 0; kb < T::kMB; ++kb) {
             const int chunk = 2 * kb + k_half;
@@ -197,8 +202,16 @@ __device__ void attend_unit(const AttendArgs& A, int u, int L, const int2* items
             uint32_t af[4];
             ldsm_x4(af, addr);
 #pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                if (kTwo && (kb & 1)) mma_bf16_16816(sacc2[nb], af, qf[kb][nb][0], qf[kb][nb][1]);
+                else mma_bf16_16816(sacc[nb], af, qf[kb][nb][0], qf[kb][nb][1]);
+            }
+        }
+        if constexpr (kTwo) {
+#pragma unroll
             for (int nb = 0; nb < NB; ++nb)
-                mma_bf16_16816(sacc[nb], af, qf[kb][nb][0], qf[kb][nb][1]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sacc[nb][i] += sacc2[nb][i];
         }
         const int t0 = page * kPage + gq, t1 = t0 + 8;
         const bool f0 = t0 < Pe || t0 >= Lw, f1 = t1 < Pe || t1 >= Lw;
@@ -287,7 +300,9 @@ __device__ void attend_unit(const AttendArgs& A, int u, int L, const int2* items
     }
     cp_async_wait<0>();
 
-    // ---- merge the warps of this CTA (Ow aliases the page buffers)
+    // ---- merge the warps of this CTA (Ow aliases the page buffers): each
+    // warp's O^T goes to Ow[warp][column][head] (the fragment pairs of two
+    // heads as one 8-byte store), m and l to ms and ls
     __syncthreads();
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
@@ -307,35 +322,50 @@ __device__ void attend_unit(const AttendArgs& A, int u, int L, const int2* items
         }
 #pragma unroll
         for (int mb = 0; mb < T::kMB; ++mb) {
-            float* ow = Ow + (size_t)warp * T::kHeads * D;
-            const int h0 = nb * 8 + 2 * tq, c0 = mb * 16 + gq;
-            ow[(size_t)h0 * D + c0] = o[mb][nb][0];
-            ow[(size_t)(h0 + 1) * D + c0] = o[mb][nb][1];
-            ow[(size_t)h0 * D + c0 + 8] = o[mb][nb][2];
-            ow[(size_t)(h0 + 1) * D + c0 + 8] = o[mb][nb][3];
+            float* ow = Ow + ((size_t)warp * D + mb * 16 + gq) * T::kHeads + nb * 8 + 2 * tq;
+            *reinterpret_cast<float2*>(ow) = make_float2(o[mb][nb][0], o[mb][nb][1]);
+            *reinterpret_cast<float2*>(ow + 8 * T::kHeads) = make_float2(o[mb][nb][2], o[mb][nb][3]);
         }
     }
     __syncthreads();
-
-    // ---- this CTA's partial record of the unit (merged by the combine kernel)
-    for (int idx = tid; idx < G * D; idx += 32 * W) {
-        const int h = idx / D, c = idx % D;
+    // per head: M = max over the warps, each warp's factor 2^(m_w - M) in
+    // place of its m, and the sum of l_w times the factor
+    if (tid < G) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < W; ++w) M = fmaxf(M, ms[w * T::kHeads + h]);
-        float acc = 0.f, lsum = 0.f;
+        for (int w = 0; w < W; ++w) M = fmaxf(M, ms[w * T::kHeads + tid]);
+        float lsum = 0.f;
 #pragma unroll
         for (int w = 0; w < W; ++w) {
-            const float mw = ms[w * T::kHeads + h];
+            const float mw = ms[w * T::kHeads + tid];
             const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
-            acc += Ow[((size_t)w * T::kHeads + h) * D + c] * f;
-            lsum += ls[w * T::kHeads + h] * f;
+            ms[w * T::kHeads + tid] = f;
+            lsum += ls[w * T::kHeads + tid] * f;
         }
-        rec[(size_t)h * D + c] = acc;
-        if (c == 0) {
-            rec[(size_t)G * D + h] = M;
-            rec[(size_t)G * D + G + h] = lsum;
+        rec[(size_t)G * D + tid] = M;
+        rec[(size_t)G * D + G + tid] = lsum;
+    }
+    __syncthreads();
+    // ---- this CTA's partial record of the unit (merged by the combine
+    // kernel): a thread sums one column of four heads over the warps
+    const int hq = (G + 3) / 4;
+    for (int idx = tid; idx < hq * D; idx += 32 * W) {
+        const int c = idx % D, h0 = 4 * (idx / D);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+            const float4 f = *reinterpret_cast<const float4*>(ms + w * T::kHeads + h0);
+            const float4 v =
+                *reinterpret_cast<const float4*>(Ow + ((size_t)w * D + c) * T::kHeads + h0);
+            acc.x += v.x * f.x;
+            acc.y += v.y * f.y;
+            acc.z += v.z * f.z;
+            acc.w += v.w * f.w;
         }
+        rec[(size_t)h0 * D + c] = acc.x;
+        if (h0 + 1 < G) rec[(size_t)(h0 + 1) * D + c] = acc.y;
+        if (h0 + 2 < G) rec[(size_t)(h0 + 2) * D + c] = acc.z;
+        if (h0 + 3 < G) rec[(size_t)(h0 + 3) * D + c] = acc.w;
     }
     __syncthreads();   // Ow / ms / ls and the page buffers are reused next
 }
