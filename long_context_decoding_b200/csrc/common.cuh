@@ -150,9 +150,14 @@ __host__ __device__ __forceinline__ SeqGeom seq_geom(int L, int prefix, int wind
 // ------------------------------------------------------------ launches
 // Launch with programmatic stream serialization: the grid may start while
 // the previous kernel on the stream is still running.  Every kernel of this
-// library therefore reads only caller inputs before pdl_wait(), and calls
-// pdl_launch_dependents() only after it, so that when a kernel starts, all
-// kernels two or more launches earlier have completed.
+// library reads only caller inputs before pdl_wait(), with two exceptions
+// that also read library-written data early: the prefix/window work of the
+// fused kernel (after the scoring kernel) and of the early decode (after the
+// selection kernel).  The kernels ahead of those two call
+// pdl_launch_dependents() only after their own wait, so that when either
+// starts, every kernel two or more launches earlier has completed.  The
+// append kernel, which neither of those two can follow, lets the next grid
+// start at its own start.
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,

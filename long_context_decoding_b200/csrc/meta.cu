@@ -187,8 +187,10 @@ __global__ void meta_update_kernel(MetaParams p) {
     const int n_touched = bad_len || L == 0 ? 0 : (L - 1) / kPage - start / kPage + 1;
     const int j0 = (int)blockIdx.y;
     const int phys0 = j0 < n_touched ? p.page_table[(size_t)b * MP + start / kPage + j0] : -1;
-    pdl_wait();
+    // the next grid may start now: whatever follows an append reads only
+    // caller inputs before its own dependency wait, which covers this kernel
     pdl_launch_dependents();
+    pdl_wait();
     if (bad_len) {
         if (c == 0 && blockIdx.y == 0) latch_flag(p.flags, CSA_DEVFLAG_BAD_SEQ_LEN);
         return;
