@@ -18,9 +18,10 @@
 //     pages' tokens outside prefix and window (a selected boundary page keeps
 //     its prefix/window tokens in the other role).  Every CTA writes one
 //     partial record of its unit (slot 8u + rank of the second record region).
-//   - prefix/window CTAs (the rest): they attend over every unit's fixed
-//     list (the pages holding prefix or window tokens, masked to those
-//     tokens), flattened and split evenly, and never wait: nothing they read
+//   - prefix/window CTAs (the rest: as many clusters as stay resident beside
+//     the selection clusters): they attend over every unit's fixed list (the
+//     pages holding prefix or window tokens, masked to those tokens),
+//     flattened and split evenly, and never wait: nothing they read
 //     is written by the scoring kernel, and by the time this grid starts the
 //     kernels before the scoring kernel (the token append among them) have
 //     finished.  They run while the scoring kernel ends and while the
