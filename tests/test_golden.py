@@ -118,4 +118,6 @@ def test_cuda_path_on_the_worked_example(one_call):
     # one bf16 rounding of an fp32 result
     np.testing.assert_allclose(o[0, :, :2], ex["expected_out"], rtol=2 ** -8, atol=1e-6)
     assert not o[0, :, 2:].any()
-    np.testing.assert_allclose(lse.cpu().numpy()[0], ex["expected_lse"], rtol=1e-5)
+    # the probabilities enter the sum of exponentials as the bf16 values the
+    # P.V product uses (each within 2^-9 relative), so lse is within ~2^-9
+    np.testing.assert_allclose(lse.cpu().numpy()[0], ex["expected_lse"], rtol=1e-4, atol=1e-3)
