@@ -123,8 +123,9 @@ typedef struct csa_dims {
 size_t csa_workspace_size(const csa_dims *d);
 
 /* Zero `bytes` of `workspace` on `stream`.  Required once before the first
- * call that uses a fresh workspace (the device flag word must start at
- * zero). */
+ * call that uses a fresh workspace: the device flag word and the per-unit
+ * key ranges that the scoring kernel merges with atomicMax must start at
+ * zero (every selection leaves its ranges at zero again). */
 int csa_workspace_init(void *workspace, size_t bytes, void *stream);
 
 /*
