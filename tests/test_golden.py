@@ -121,3 +121,48 @@ def test_cuda_path_on_the_worked_example(one_call):
     # the probabilities enter the sum of exponentials as the bf16 values the
     # P.V product uses (each within 2^-9 relative), so lse is within ~2^-9
     np.testing.assert_allclose(lse.cpu().numpy()[0], ex["expected_lse"], rtol=1e-4, atol=1e-3)
+
+
+def test_oracle_fp8_copy_on_the_worked_example():
+    """Every key of the example (0, +-1, 0.5) is a power of two times an E4M3
+    value, so the fp8 copy holds the exact box and its scores are the exact
+    ones."""
+    ex = load()
+    q, k, v, pt, sl = build(ex)
+    d = oracle.Dims(1, 2, 1, D, ex["page_size"], pt.shape[1], pt.shape[1])
+    m8 = oracle.meta_fp8(d, oracle.meta(d, k, pt, sl), pt, sl)
+    sc = oracle.scores_fp8(d, q, m8, pt, sl, ex["prefix"], ex["window"])
+    for page, want in ex["expected_scores"].items():
+        assert sc[0, 0, int(page)] == want
+
+
+@pytest.mark.gpu
+def test_cuda_fp8_path_on_the_worked_example():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_decoding_b200 import csa
+    ex = load()
+    q, k, v, pt, sl = build(ex)
+    dev = torch.device("cuda:0")
+    t = lambda a, dt: torch.from_numpy(a.astype(dt)).to(dev)
+    qd = t(q, np.int16).view(torch.bfloat16)
+    kd = t(k, np.int16).view(torch.bfloat16)
+    vd = t(v, np.int16).view(torch.bfloat16)
+    ptd, sld = t(pt, np.int32), t(sl, np.int32)
+    n_pages = pt.shape[1]
+    d = csa.make_dims(1, 2, 1, D, n_pages, n_pages, 4)
+    lay = csa.Layer(d, kd, vd, ptd, sld, ex["prefix"], ex["window"], ex["budget"], fp8=True)
+    lay.rebuild_meta()
+    sel = torch.full((1, 1, 4), -7, dtype=torch.int32, device=dev)
+    nsel = torch.full((1, 1), -7, dtype=torch.int32, device=dev)
+    out = torch.empty((1, 2, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((1, 2), dtype=torch.float32, device=dev)
+    csa.sparse_attention_fp8(d, qd, kd, vd, lay.meta8, ptd, sld, ex["prefix"], ex["window"],
+                             ex["budget"], sel, nsel, out, lay.ws, lse, scale=1.0)
+    torch.cuda.synchronize()
+    assert csa.device_status(lay.ws) == 0
+    assert nsel[0, 0].item() == len(ex["expected_selection"])
+    assert sel[0, 0, :nsel[0, 0].item()].tolist() == ex["expected_selection"]
+    o = out.float().cpu().numpy()
+    np.testing.assert_allclose(o[0, :, :2], ex["expected_out"], rtol=2 ** -8, atol=1e-6)
+    np.testing.assert_allclose(lse.cpu().numpy()[0], ex["expected_lse"], rtol=1e-4, atol=1e-3)
