@@ -66,6 +66,8 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=0,
                     help="use only the first N layers (small cases for ncu captures)")
     ap.add_argument("--no-fp8", action="store_true", help="skip the fp8-metadata line")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the compact sparse-vs-dense sweep of the default run")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the step: sparse (one call) vs dense decode over uniform "
                          "lengths 4k..256k and budgets 0/1024/4096/all, with a byte-based "
@@ -135,6 +137,26 @@ def score_traffic():
         return rec["dram_bytes_per_launch"], rec["workload"]
     except Exception:
         return None, None
+
+
+def step_dram_traffic():
+    """DRAM bytes per 256k layer step (all kernels of one append +
+    csa_sparse_attention) from the committed ncu launch summary, or None
+    when a kernel source changed since those counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic_layer_step.txt")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for name in sorted(rec["sources"]):
+            with open(os.path.join(ROOT, "long_context_decoding_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["sources_sha256"]:
+            return None
+        return {"bytes_per_layer_step": rec["dram_bytes_per_layer_step"],
+                "source": rec["source"]}
+    except Exception:
+        return None
 
 
 def hbm_peak():
@@ -307,16 +329,18 @@ class Stack:
     def launches_per_step(self) -> int:
         """Kernels of one step: per layer the metadata update, then the scoring
         kernel, the fused selection + decode kernel and the split-K combine
-        when the one-call path applies (k >= 1, at most 32 units, at most
-        16384 candidates per unit), else scoring (k >= 1), selection, decode
-        and combine."""
+        when the one-call path applies (1 <= k < candidates, at most 32 units,
+        at most 16384 candidates per unit), else scoring (when k chooses),
+        selection, decode and combine."""
         w = self.w
         n = 0
         for lay in self.layers:
             k = lay.budget // 16
             n_max = w.max_pages - lay.prefix // 16 - lay.window // 16
-            fused = k > 0 and w.B * w.Hkv <= 32 and n_max <= 16384
-            n += 1 + (3 if fused else (1 if k > 0 else 0) + 3)
+            if 0 < k < n_max and n_max <= 16384 and w.B * w.Hkv <= 32:
+                n += 1 + 3
+            else:   # selection (or the full list), decode, combine; scores when k chooses
+                n += 1 + (1 if 0 < k < n_max else 0) + 3
         return n
 
     def graph(self, fn):
@@ -447,17 +471,28 @@ def run_ours(args, dist: Dist, base: wl.Workload):
                             "gbs": dec_bytes / times["decode"] / 1e9}}
         ach = calls["score"]["gbs"]
         traffic, traffic_src = score_traffic()
-        line["roofline"] = {"bound": "hbm", "kernel": "score_direct_kernel (Quest scoring)",
-                            "achieved": ach, "peak": peak, "peak_kind": peak_kind,
-                            "unit": "GB/s", "frac": ach / peak, "traffic": traffic,
-                            "traffic_source": (f"ncu dram__bytes_read+write per launch, {traffic_src}, "
-                                               "profiles/score_kernel_ctx256k_layer.md")
-                                              if traffic else None,
-                            "note": "dominant kernel at 256k (largest share of the ncu launch "
-                                    "list); achieved = metadata bytes of the candidate pages "
-                                    "(|C| x 4D per unit) / CUDA-event time per call, from graph "
-                                    "replays of budget-0 csa_score_select calls over the 12 "
-                                    "layers (scoring kernel + an empty selection launch)"}
+        step_ach = layer_sparse / t_layer / 1e9
+        step_traffic = step_dram_traffic()
+        line["roofline"] = {
+            "bound": "hbm", "scope": "layer step",
+            "achieved": step_ach, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+            "frac": step_ach / peak, "frac_of_8tbs_nominal": step_ach / NOMINAL_HBM_GBS,
+            "traffic": step_traffic["bytes_per_layer_step"] if step_traffic else None,
+            "traffic_source": step_traffic["source"] if step_traffic else None,
+            "note": "achieved = algorithmic bytes of a layer step (metadata of the candidate "
+                    "pages + K/V of the attended tokens + q/out; mean over the 12 layers and "
+                    "the timed steps) / device time of a layer step (append + "
+                    "csa_sparse_attention: scoring, selection, attention, combine) from the "
+                    "timed graph replays",
+            "kernel": "score_direct_kernel (Quest scoring; the largest share of the launch list)",
+            "kernel_achieved": ach, "kernel_frac": ach / peak, "kernel_traffic": traffic,
+            "kernel_traffic_source": (f"ncu dram__bytes_read+write per launch, {traffic_src}, "
+                                      "profiles/score_kernel_ctx256k_layer.md")
+                                     if traffic else None,
+            "kernel_note": "metadata bytes of the candidate pages (|C| x 4D per unit) / "
+                           "CUDA-event time per call, from graph replays of budget-0 "
+                           "csa_score_select calls over the 12 layers (scoring kernel + an "
+                           "empty selection launch)"}
         line["calls"] = calls
         line["clocks"] = clk
 
@@ -473,6 +508,10 @@ def run_ours(args, dist: Dist, base: wl.Workload):
         if not args.no_secondary and base.name == wl.CTX256K.name:
             line["ctx64k"] = secondary_64k(dev, dist)
 
+        # ---- sparse against dense over context length, and the cost model
+        if not args.no_sweep and base.name == wl.CTX256K.name:
+            line["sweep"] = compact_sweep(dev, dist)
+
         # ---- CPU oracle on a bounded sample
         if not args.no_cpu_baseline and dist.rank == 0 and dist.world == 1:
             rate, n, el, threads, sample = oracle_sample(base, args.cpu_seconds)
@@ -482,6 +521,13 @@ def run_ours(args, dist: Dist, base: wl.Workload):
                                     "kind": "oracle", "sample": sample,
                                     "one_core": {"value": r1, "cores": 1, "sample": s1},
                                     "dense": {"value": rd, "cores": td, "sample": sd}}
+            if not args.no_secondary and base.name == wl.CTX256K.name:
+                rec = oracle_planted_recall(dev)
+                line["cpu_baseline"]["planted_recall_oracle"] = {
+                    "workload": wl.CTX64K.name, "mean": rec["mean"], "min": rec["min"],
+                    "per_unit": rec["per_unit"],
+                    "note": "the oracle's top-k on the same seeded 64k inputs: the fraction of "
+                            "the 32 planted pages per (sequence, kv-head) it selects"}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -615,13 +661,53 @@ def secondary_64k(dev, dist: Dist):
     out = torch.empty_like(lay.out)
     tdn = graph_time(lambda: csa.decode_full(d, c.q, c.k_cache, c.v_cache, c.page_table,
                                              c.seq_lens, out, lay.ws), 10, 3, flush)
+    lay.step(c.q, fused=True)
+    recall = planted_recall(lay.sel.cpu().numpy(), lay.n_sel.cpu().numpy(),
+                            c.planted_pages.cpu().numpy())
     return {"workload": w.name, "value": dist.world * w.B / t, "unit": UNIT,
             "us_per_layer_step": 1e6 * t, "algorithmic_bytes": by["sparse"],
+            "frac": ach / peak,
+            "planted_recall": {"mean": recall["mean"], "min": recall["min"],
+                               "per_unit": recall["per_unit"],
+                               "note": "fraction of the 32 q-aligned planted pages per "
+                                       "(sequence, kv-head) that the one-call selection holds "
+                                       "(a measurement; the oracle's own figure is in "
+                                       "cpu_baseline.planted_recall_oracle)"},
             "achieved_gbs": ach, "frac_of_measured_peak": ach / peak,
             "frac_of_8tbs_nominal": ach / NOMINAL_HBM_GBS,
             "dense_us": 1e6 * tdn, "dense_gbs": by["dense"] / tdn / 1e9,
             "speedup_vs_dense": tdn / t,
             "timing": "batches of 20 graph replays, each after a 256 MB L2 flush (read); the flush time subtracted; median of 3 batches"}
+
+
+def planted_recall(sel, nsel, planted):
+    """Per (sequence, kv-head): the fraction of its planted pages that the
+    selection sel[b][g][:nsel[b][g]] holds."""
+    per = []
+    for b in range(planted.shape[0]):
+        for g in range(planted.shape[1]):
+            got = set(int(x) for x in sel[b, g, :int(nsel[b, g])])
+            want = [int(x) for x in planted[b, g]]
+            per.append(sum(p in got for p in want) / len(want))
+    return {"mean": sum(per) / len(per), "min": min(per), "per_unit": per}
+
+
+def oracle_planted_recall(dev):
+    """The oracle's selection on the 64k planted workload (same seeded
+    inputs, copied to the host) and its planted-page recall."""
+    import oracle
+    w = wl.CTX64K
+    c = wl.make_case(w, dev)
+    d = oracle.Dims(w.B, w.Hq, w.Hkv, w.D, 16, w.max_pages, w.num_pages)
+    q, k = wl.bits(c.q), wl.bits(c.k_cache)
+    pt, sl = c.page_table.cpu().numpy(), c.seq_lens.cpu().numpy()
+    planted = c.planted_pages.cpu().numpy()
+    del c
+    torch.cuda.empty_cache()
+    oracle.set_threads(len(os.sched_getaffinity(0)))
+    sc = oracle.scores(d, q, k, pt, sl, w.prefix, w.window)
+    sel, nsel = oracle.select(d, sc, sl, w.prefix, w.window, w.budget, w.max_sel)
+    return planted_recall(sel, nsel, planted)
 
 
 def graph_time(fn, reps: int, warm: int, flush) -> float:
@@ -657,16 +743,13 @@ def graph_time(fn, reps: int, warm: int, flush) -> float:
     return statistics.median((batch(True) - batch(False)) / reps for _ in range(3))
 
 
-def run_sweep(args, dist: Dist):
+def sweep_points(dev, grid, budgets, reps: int, warm: int):
     """Sparse (csa_sparse_attention) against dense (csa_decode_full) decode on
     the same cache, batch 4, 16 query / 4 kv heads, D 128, prefix 128, window
-    1024, at every length of the sweep grid and every budget; then the cost
-    model t = t0 + bytes / bw fitted to the sparse points by least squares."""
+    1024, at every length of `grid` and every budget of `budgets` (None: the
+    whole context); each time from graph replays with L2 flushed (graph_time).
+    Returns the points and the cost-model fits over them."""
     from long_context_decoding_b200 import csa
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py: no CUDA device (the CUDA path has no CPU fallback)")
-    dev = torch.device("cuda", dist.local)
-    torch.cuda.set_device(dev)
     scrub = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MB
     sink = torch.zeros((), device=dev)
 
@@ -674,7 +757,7 @@ def run_sweep(args, dist: Dist):
         torch.sum(scrub, dim=0, out=sink)
 
     points = []
-    for L in wl.SWEEP_GRID:
+    for L in grid:
         w = replace(wl.SWEEP, name=f"b4_h16x4_d128_ctx{L}", seq_lens=(L,) * 4)
         c = wl.make_case(w, dev)
         d = csa.make_dims(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.num_pages, w.max_pages)
@@ -684,10 +767,10 @@ def run_sweep(args, dist: Dist):
         out = torch.empty_like(lay.out)
         t_dense = graph_time(lambda: csa.decode_full(d, c.q, c.k_cache, c.v_cache,
                                                        c.page_table, c.seq_lens, out, lay.ws),
-                               args.steps, args.warmup, flush)
-        for budget in wl.SWEEP_BUDGETS:
+                               reps, warm, flush)
+        for budget in budgets:
             lay.budget = PS_TOKENS * w.max_pages if budget is None else budget
-            t = graph_time(lambda: lay.step(c.q, fused=True), args.steps, args.warmup, flush)
+            t = graph_time(lambda: lay.step(c.q, fused=True), reps, warm, flush)
             by = cost.layer_bytes(w.seq_lens, w.Hq, w.Hkv, w.D, w.prefix, w.window, budget)
             points.append({"L": L, "budget": "all" if budget is None else budget,
                            "path": cost.path_of(L, w.prefix, w.window, budget),
@@ -697,7 +780,7 @@ def run_sweep(args, dist: Dist):
         assert csa.device_status(lay.ws) == 0
         del c, lay, out
         torch.cuda.empty_cache()
-    # cost model over the sparse points
+    # one fixed cost for every point
     x = [p["sparse_bytes"] for p in points]
     y = [p["sparse_us"] * 1e-6 for p in points]
     n = len(x)
@@ -707,6 +790,41 @@ def run_sweep(args, dist: Dist):
     for p in points:
         p["model_us"] = 1e6 * (t0 + slope * p["sparse_bytes"])
     worst = max(abs(p["model_us"] - p["sparse_us"]) / p["sparse_us"] for p in points)
+    per_path = cost.fit_per_path(points)
+    for p in points:
+        p["model_per_path_us"] = (per_path["t0_us"][p["path"]]
+                                  + p["sparse_bytes"] / (per_path["bw_gbs"] * 1e3))
+    fits = {"cost_model": {"t0_us": 1e6 * t0, "bw_gbs": 1.0 / slope / 1e9, "max_rel_err": worst,
+                           "form": "t = t0 + algorithmic bytes / bw"},
+            "cost_model_per_path": per_path}
+    return points, fits
+
+
+def compact_sweep(dev, dist: Dist):
+    """The sweep's key points for the default run: sparse against dense at
+    16k, 32k, 64k and 256k for budgets 0, 1024 and 4096, with the per-path
+    cost-model fit over them."""
+    points, fits = sweep_points(dev, (16384, 32768, 65536, 262144), (0, 1024, 4096), 10, 3)
+    keep = ("L", "budget", "path", "sparse_us", "dense_us", "speedup", "sparse_gbs",
+            "model_per_path_us")
+    return {"config": "batch 4, 16 query / 4 kv heads, D 128, prefix 128, window 1024, uniform "
+                      "lengths; csa_sparse_attention against csa_decode_full on the same cache; "
+                      "graph replays after a 256 MB L2 read-flush, median of 3 batches",
+            "points": [{k: p[k] for k in keep} for p in points],
+            "sparse_faster_than_dense_for_all_L_ge_32k":
+                all(p["sparse_us"] < p["dense_us"] for p in points if p["L"] >= 32768),
+            "cost_model_per_path": fits["cost_model_per_path"]}
+
+
+def run_sweep(args, dist: Dist):
+    """The full sweep (--sweep): every length of the grid, budgets 0, 1024,
+    4096 and all; the cost model t = t0 + bytes / bw fitted by least squares,
+    with one fixed cost and with one per path."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the CUDA path has no CPU fallback)")
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    points, fits = sweep_points(dev, wl.SWEEP_GRID, wl.SWEEP_BUDGETS, args.steps, args.warmup)
     # a budget of "all" attends to every token: the same work as dense
     beats = all(p["sparse_us"] < p["dense_us"] for p in points
                 if p["L"] >= 32768 and p["budget"] != "all")
@@ -718,10 +836,7 @@ def run_sweep(args, dist: Dist):
                        "q_heads": 16, "kv_heads": 4, "head_dim": 128, "prefix": 128,
                        "window": 1024, "l2": "256 MB read between replays",
                        "timing": "median of graph replays, CUDA events"},
-            "points": points,
-            "cost_model": {"t0_us": 1e6 * t0, "bw_gbs": 1.0 / slope / 1e9,
-                           "max_rel_err": worst, "form": "t = t0 + algorithmic bytes / bw"},
-            "cost_model_per_path": cost.fit_per_path(points),
+            "points": points, **fits,
             "sparse_faster_than_dense_for_all_L_ge_32k": beats,
             "all_budget_min_speedup_vs_dense": all_ratio}
     if dist.rank == 0:

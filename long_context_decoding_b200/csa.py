@@ -18,6 +18,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcsa.so")
 
 CSA_OK = 0
+CSA_ERR_INVALID_ARG = -1
+CSA_ERR_UNSUPPORTED = -2
+CSA_ERR_WORKSPACE = -3
+CSA_ERR_CUDA = -4
 CSA_ERR_DEVICE_FLAG = -5
 DEVFLAG_BAD_PAGE_ID = 1
 DEVFLAG_BAD_SELECTION = 2

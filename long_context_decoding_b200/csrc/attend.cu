@@ -179,17 +179,16 @@ __global__ void __cluster_dims__(kCl, 1, 1)
     pdl_launch_dependents();
 
     if (kk == n) {              // every candidate fits the budget
-        for (int j = lo + tid; j < hi; j += kClThreads) {
-            share[j - lo] = c_lo + j;
-            out[j] = c_lo + j;
-        }
+        for (int j = lo + tid; j < hi; j += kClThreads) share[j - lo] = c_lo + j;
     } else if (kk > 0) {
         uint32_t kmin, kmax;
         key_range(P.keyrange[u], kmin, kmax);
+        // only shared-memory stores before the barrier (its release then
+        // waits for no global store); each CTA writes its share of the
+        // output list afterwards
         cluster_select(cl, sh, P.scores_ws + (size_t)u * MP + c_lo, n, kk, kmin, kmax,
                        [&](int pos, int i) {
-                           out[pos] = c_lo + i;
-                           const int dst = cta_of(pos, kk, kCl);
+                           const int dst = ((pos + 1) * kCl + kk - 1) / kk - 1;
                            int* d = cl.map_shared_rank(share, dst);
                            d[pos - kk * dst / kCl] = c_lo + i;
                        });
@@ -204,6 +203,7 @@ __global__ void __cluster_dims__(kCl, 1, 1)
     const int cnt = hi - lo;
     for (int j = tid; j < cnt; j += kClThreads) {
         const int page = share[j];
+        out[lo + j] = page;
         int phys = p.page_table[(size_t)b * MP + page];
         if (phys < 0 || phys >= p.s.NPG) {
             latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);

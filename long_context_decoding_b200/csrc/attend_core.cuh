@@ -94,7 +94,7 @@ __device__ __forceinline__ int cta_of(long long x, long long T, int n) {
 // Partial record of one (CTA, unit): o[G][D] relative to the CTA's own max,
 // then m[G] (max, exp2 domain) and l[G] (sum); the stride keeps o 16-byte
 // aligned.
-__host__ __device__ __forceinline__ size_t record_stride(int G, int D) {
+__host__ __device__ constexpr __forceinline__ size_t record_stride(int G, int D) {
     return ((size_t)G * D + 2 * G + 3) & ~(size_t)3;
 }
 

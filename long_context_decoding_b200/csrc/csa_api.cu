@@ -80,7 +80,7 @@ WsLayout workspace_layout(const Shape& s) {
 // ---------------------------------------------------------------- validation
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-static int check_dims(const csa_dims* d, Shape* s) {
+int check_dims(const csa_dims* d, Shape* s) {
     if (!d) return CSA_ERR_INVALID_ARG;
     if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->D < 1 || d->max_pages_per_seq < 1 ||
         d->num_pages < 1 || d->max_sel < 1)
@@ -363,6 +363,8 @@ static int sparse_attention_common(const csa_dims* d, const void* q, const void*
     if (rc != CSA_OK) return rc;
     cudaStream_t st = (cudaStream_t)stream;
     note_stream_call(stream, kCallOther);
+    const long long n_max = (long long)s.MP - prefix / kPage - window / kPage;
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)s.D);
 
     ScoreParams sp;
     sp.q = static_cast<const uint16_t*>(q);
@@ -377,7 +379,6 @@ static int sparse_attention_common(const csa_dims* d, const void* q, const void*
     sp.keyrange = at<uint2>(workspace, w.keyrange);
     sp.flags = at<uint32_t>(workspace, w.flags);
     sp.s = s;
-    const long long n_max = (long long)s.MP - prefix / kPage - window / kPage;
     if (k_pages > 0 && k_pages < n_max) {      // else every unit keeps all its candidates
         rc = launch_status(launch_score(sp, st));
         if (rc != CSA_OK) return rc;
@@ -394,7 +395,6 @@ static int sparse_attention_common(const csa_dims* d, const void* q, const void*
     dp.prefix = prefix;
     dp.window = window;
     dp.dense = 0;
-    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)s.D);
     dp.scale_log2 = sc * 1.4426950408889634f;
     dp.out = static_cast<uint16_t*>(out);
     dp.lse = lse;

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/csa.h"
+
 namespace csa {
 
 // Workspace layout (byte offsets into the caller's workspace).
@@ -127,6 +129,10 @@ cudaError_t launch_shard_selection(const Shape& s, const int32_t* sel, const int
                                    int32_t* n_local, cudaStream_t st);
 cudaError_t launch_merge(int parts, int bh_count, int D, const void* out_parts,
                          const float* lse_parts, void* out, float* lse, cudaStream_t st);
+
+// Validates a csa_dims (sizes, supported head dims and group sizes, index
+// ranges) and fills the kernel-side shape; CSA_OK or the status to return.
+int check_dims(const ::csa_dims* d, Shape* s);
 
 int device_sm_count();
 int decode_grid(const Shape& s);

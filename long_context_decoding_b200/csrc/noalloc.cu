@@ -67,30 +67,13 @@ extern "C" int csa_decode_noalloc(const csa_dims* d, const void* q, const void* 
                                   const int32_t* seq_lens, const int32_t* sel_pages,
                                   const int32_t* n_sel, int prefix, int window, float scale,
                                   void* out, float* lse, void* stream) {
-    if (!d || d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->max_pages_per_seq < 1 ||
-        d->num_pages < 1 || d->max_sel < 1 || d->Hq % d->Hkv != 0)
-        return CSA_ERR_INVALID_ARG;
-    const int G = d->Hq / d->Hkv;
-    if (d->page_size != kPage || (d->D != 64 && d->D != 128 && d->D != 256) ||
-        (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) ||
-        (long long)d->B * d->Hkv > kMaxUnits ||
-        (long long)d->num_pages * d->Hkv * kPage >= (1ll << 31) ||
-        (long long)d->max_pages_per_seq * kPage >= (1ll << 31))
-        return CSA_ERR_UNSUPPORTED;
+    Shape s;
+    const int rc = check_dims(d, &s);
+    if (rc != CSA_OK) return rc;
     if (!ok16(q) || !ok16(k_cache) || !ok16(v_cache) || !ok16(page_table) || !ok16(seq_lens) ||
         !ok16(sel_pages) || !ok16(n_sel) || !ok16(out) || (lse && !ok16(lse)))
         return CSA_ERR_INVALID_ARG;
     if (prefix < 0 || window < 0 || !(scale == scale) || isinf(scale)) return CSA_ERR_INVALID_ARG;
-
-    Shape s;
-    s.B = d->B;
-    s.Hq = d->Hq;
-    s.Hkv = d->Hkv;
-    s.G = G;
-    s.D = d->D;
-    s.MP = d->max_pages_per_seq;
-    s.NPG = d->num_pages;
-    s.max_sel = d->max_sel;
 
     // scratch: [flag word | record ranges | partial records of the two
     // decode phases], each 256-byte aligned

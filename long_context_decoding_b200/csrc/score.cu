@@ -66,12 +66,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
         : "r"(w));
     return h2;
 }
-// bf16x2 -> f16x2 (exact for |x| in [2^-17, 65504]; larger values saturate).
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
-    uint32_t r;
-    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(bf16_hi(w)), "f"(bf16_lo(w)));
-    return r;
-}
 
 // 16-byte load that does not allocate in L1 (the metadata is read once).
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
@@ -397,8 +391,12 @@ struct RingCfg {
 // gives lane (g, t) the four channels 4t .. 4t+3 of row g's 16-channel chunk;
 // the hardware converts each pair to f16 (exact), the pairs become the k
 // slots (2t, 2t+1) and (2t+8, 2t+9) of an f16 MMA whose q side takes the same
-// channels, q is converted to f16 (exact for |q| >= 2^-17), and the row's sums
-// are scaled by 2^e.
+// channels.  Each head's q is scaled by 2^-f, f chosen so that its largest
+// component lands in [2^14, 2^15), and converted to f16: exact for every
+// component within 2^-31 of the head's largest (the rest, which move the sum
+// by less than its fp32 rounding, round to the f16 grid), and never
+// saturated, whatever the magnitude of q.  The row's sums are scaled back by
+// 2^(e + f), exactly.
 template <int D, int NB, bool F8>
 __global__ void __launch_bounds__(RingCfg<D, F8>::kThreads, 2)
 score_ring_kernel(ScoreParams p) {
@@ -448,6 +446,7 @@ score_ring_kernel(ScoreParams p) {
     // B fragments of [q- | q+] for the current unit: MMA kk covers the 16
     // channels [16 kk, 16 kk + 16) of the [min | max] row (min pairs with q-)
     uint32_t qf[D / 8][NB][2];
+    int qexp[NB][2];       // F8: exponent f of the heads of accumulator columns 2t, 2t + 1
     int cur_unit = -1;
     KeyRange kr;
 
@@ -469,9 +468,40 @@ score_ring_kernel(ScoreParams p) {
                         const int ch = F8 ? 16 * kk + 4 * tq + 2 * h : 16 * kk + 8 * h + 2 * tq;
                         const int qc = is_max ? ch - D : ch;
                         const uint32_t v = head < G ? __ldg(qw + qc / 2) : 0u;
-                        const uint32_t part = is_max ? pos_part(v) : neg_part(v);
-                        qf[kk][nb][h] = F8 ? bf16x2_to_f16x2(part) : part;
+                        qf[kk][nb][h] = is_max ? pos_part(v) : neg_part(v);
                     }
+                }
+            }
+            if constexpr (F8) {
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    // largest |q| of head nb * 8 + g: this lane holds a quarter
+                    // of its channels (each once in the q- and once in the q+ half)
+                    float amax = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < D / 8; ++kk)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(qf[kk][nb][h])),
+                                                     fabsf(bf16_hi(qf[kk][nb][h]))));
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                    const int f = amax > 0.f ? ilogbf(amax) - 14 : 0;
+#pragma unroll
+                    for (int kk = 0; kk < D / 8; ++kk)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t w = qf[kk][nb][h];
+                            uint32_t r;
+                            asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;"
+                                : "=r"(r)
+                                : "f"(ldexpf(bf16_hi(w), -f)), "f"(ldexpf(bf16_lo(w), -f)));
+                            qf[kk][nb][h] = r;
+                        }
+                    // accumulator columns 2t and 2t + 1 belong to the heads
+                    // loaded by the lanes with g = 2t and g = 2t + 1
+                    qexp[nb][0] = __shfl_sync(0xffffffffu, f, 8 * tq);
+                    qexp[nb][1] = __shfl_sync(0xffffffffu, f, 8 * tq + 4);
                 }
             }
         }
@@ -513,15 +543,14 @@ score_ring_kernel(ScoreParams p) {
                 }
             }
             const uint8_t* rows = ring + stage * C::kTileSmem;
-            const float sc0 = ldexpf(1.f, *reinterpret_cast<const int*>(rows + gq * C::kStride + 2 * D));
-            const float sc8 =
-                ldexpf(1.f, *reinterpret_cast<const int*>(rows + (gq + 8) * C::kStride + 2 * D));
+            const int e0 = *reinterpret_cast<const int*>(rows + gq * C::kStride + 2 * D);
+            const int e8 = *reinterpret_cast<const int*>(rows + (gq + 8) * C::kStride + 2 * D);
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-                acc[nb][0] = (acc[nb][0] + acc2[nb][0]) * sc0;
-                acc[nb][1] = (acc[nb][1] + acc2[nb][1]) * sc0;
-                acc[nb][2] = (acc[nb][2] + acc2[nb][2]) * sc8;
-                acc[nb][3] = (acc[nb][3] + acc2[nb][3]) * sc8;
+                acc[nb][0] = ldexpf(acc[nb][0] + acc2[nb][0], e0 + qexp[nb][0]);
+                acc[nb][1] = ldexpf(acc[nb][1] + acc2[nb][1], e0 + qexp[nb][1]);
+                acc[nb][2] = ldexpf(acc[nb][2] + acc2[nb][2], e8 + qexp[nb][0]);
+                acc[nb][3] = ldexpf(acc[nb][3] + acc2[nb][3], e8 + qexp[nb][1]);
             }
         }
         int p0, p8;

@@ -99,10 +99,14 @@ CTX256K = Workload("b4_h32x4_d128_ctx256k_12layer", B=4, Hq=32, Hkv=4, D=128,
 SWEEP = Workload("b4_h16x4_d128_ragged4k_256k", B=4, Hq=16, Hkv=4, D=128,
                  seq_lens=_ragged(4, 4096, 262144, 0), prefix=128, window=1024,
                  budget=4096)
+# A larger batch of the 64k decode (another size of the model family): 8
+# sequences x 8 kv-heads = 64 (sequence, kv-head) units, D = 128.
+CTX64K_B8 = Workload("b8_h64x8_d128_ctx64k", B=8, Hq=64, Hkv=8, D=128,
+                     seq_lens=(65536,) * 8, prefix=128, window=2048, budget=4096)
 SWEEP_BUDGETS = (0, 1024, 4096, None)      # None = the whole context ("all")
 SWEEP_GRID = (4096, 8192, 16384, 32768, 65536, 131072, 262144)
 
-WORKLOADS = {w.name: w for w in (TINY, CTX32K, CTX64K, CTX256K, SWEEP)}
+WORKLOADS = {w.name: w for w in (TINY, CTX32K, CTX64K, CTX256K, SWEEP, CTX64K_B8)}
 
 
 @dataclass

@@ -1,7 +1,8 @@
 """GPU parity of the optional fp8 metadata path against the oracle's fp8
 definition (csa_oracle.c): the fp8 copy bit-exact (after a rebuild and after
 appends), scores to fp32 accuracy, the selection by the band rule, and the
-one-call output in every unit whose selection is the oracle's own."""
+one-call output of every unit against the oracle's attention over that unit's
+selection (the oracle's own, or the GPU's valid pick inside a tie band)."""
 import math
 from dataclasses import replace
 
@@ -12,7 +13,8 @@ import torch
 import oracle
 from long_context_decoding_b200 import csa
 from long_context_decoding_b200 import workloads as wl
-from parity import PS, assert_out_close, assert_scores_close, check_selection
+from parity import (PS, assert_out_close, assert_scores_close, check_selection,
+                    oracle_on_valid_choice)
 
 pytestmark = pytest.mark.gpu
 
@@ -80,16 +82,14 @@ def check_fp8(run: Fp8Run, one_call=True):
     gs, gn = lay.sel.cpu().numpy(), lay.n_sel.cpu().numpy()
     assert all(np.array_equal(gs[b, g, :gn[b, g]], sel_s.cpu().numpy()[b, g, :gn[b, g]])
                for b in range(run.d.B) for g in range(run.d.Hkv))
+    exp_out, exp_lse, same = oracle_on_valid_choice(run.od, h, w.prefix, run.c.window,
+                                                     1.0 / math.sqrt(w.D), lay.sel, lay.n_sel,
+                                                     ref)
     G = w.Hq // w.Hkv
-    same = 0
     for b in range(run.d.B):
         for g in range(run.d.Hkv):
-            k = int(gn[b, g])
-            if not np.array_equal(gs[b, g, :k], ref["sel"][b, g, :k]):
-                continue
-            same += 1
             hh = slice(g * G, (g + 1) * G)
-            assert_out_close(out[b, hh], lay.lse[b, hh], ref["out"][b, hh], ref["lse"][b, hh],
+            assert_out_close(out[b, hh], lay.lse[b, hh], exp_out[b, hh], exp_lse[b, hh],
                              f"fp8 one-call, unit ({b},{g})")
     return same
 
@@ -143,3 +143,46 @@ def test_fp8_scores_bound_the_bf16_scores(cuda):
     assert torch.equal(cand, ~torch.isnan(s8))
     # fp32 sums of exact products: allow their rounding
     assert (s8[cand] >= s16[cand] - 1e-5 * s16[cand].abs() - 1e-3).all()
+
+
+def test_fp8_scores_for_extreme_query_magnitudes(cuda):
+    """Query components far below 2^-17 and far above the f16 range (65504),
+    per head and mixed within one head: the scores from the fp8 copy still
+    match the oracle's fp8 definition (exact bf16 q, fp64), relative to each
+    unit's own magnitude, and the selection follows the band rule."""
+    w = wl.Workload("fp8_qrange", B=2, Hq=16, Hkv=4, D=128, seq_lens=(3000, 2049), prefix=40,
+                    window=100, budget=480, seed=17)
+    case = wl.make_case(w, cuda)
+    G = w.G
+    chan = torch.arange(w.D, device=cuda, dtype=torch.float32)
+    q = case.q.float()
+    q[:, 0 * G:1 * G] *= 2.0 ** -30                          # every component tiny
+    q[:, 1 * G:2 * G] *= 2.0 ** 24                           # beyond f16's largest value
+    q[:, 2 * G:3 * G] *= torch.exp2(chan % 64 - 44.0)        # 2^-44 .. 2^19 within each head
+    case.q = q.to(torch.bfloat16)                            # kv-head 3 as drawn
+    run = Fp8Run(case)
+    h = run.host()
+    assert_meta8_equal(run, h)
+    m8 = run.oracle_meta8(h)
+    ref = oracle.scores_fp8(run.od, h["q"], m8, h["pt"], h["sl"], w.prefix, case.window)
+    lay = run.layer
+    sc = torch.full((run.d.B, run.d.Hkv, run.d.max_pages_per_seq), float("nan"),
+                    dtype=torch.float32, device=cuda)
+    csa.score_select_fp8(run.d, case.q, lay.meta8, case.page_table, case.seq_lens, w.prefix,
+                         case.window, run.budget, lay.sel, lay.n_sel, lay.ws, scores_out=sc)
+    torch.cuda.synchronize()
+    assert csa.device_status(lay.ws) == 0
+    got = sc.cpu().numpy().astype(np.float64)
+    cand = ~np.isnan(ref)
+    assert np.array_equal(~np.isnan(got), cand)
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            c = cand[b, g]
+            r, x = ref[b, g][c], got[b, g][c]
+            scale = np.abs(r).max()
+            assert scale > 0 and np.isfinite(x).all(), f"unit ({b},{g})"
+            np.testing.assert_allclose(x, r, rtol=2e-5, atol=1e-6 * scale,
+                                       err_msg=f"fp8 scores, unit ({b},{g})")
+    sel, nsel = oracle.select(run.od, ref, h["sl"], w.prefix, case.window, run.budget,
+                              run.max_sel)
+    check_selection(lay.sel, lay.n_sel, ref, sel, nsel, gpu_scores=sc)

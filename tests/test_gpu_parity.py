@@ -12,7 +12,7 @@ import oracle
 from long_context_decoding_b200 import csa
 from long_context_decoding_b200 import workloads as wl
 from parity import (Run, assert_meta_equal, assert_out_close, assert_scores_close,
-                    check_selection)
+                    check_selection, oracle_on_valid_choice)
 
 pytestmark = pytest.mark.gpu
 PS = 16
@@ -247,8 +247,11 @@ def sparse_call(run: Run):
 
 def check_one_call(run: Run, oracle_too=True):
     """The one-call path selects exactly what csa_score_select selects, attends
-    like csa_decode on that selection, and, where the oracle's selection is
-    unambiguous for every unit, matches the oracle."""
+    like csa_decode on that selection, and matches the oracle: the selection
+    by the band rule, and the output of every unit against the oracle's
+    attention over that unit's selection (the oracle's own, or, inside a tie
+    band, the GPU's valid pick).  Returns the number of units whose selection
+    is the oracle's own."""
     run.gpu_meta()
     sel_f, nsel_f, out_f, lse_f = sparse_call(run)
     run.gpu_select(scores=False)
@@ -267,25 +270,20 @@ def check_one_call(run: Run, oracle_too=True):
     fin = torch.isfinite(lse_s)
     assert torch.equal(torch.isfinite(lse_f), fin)
     torch.testing.assert_close(lse_f[fin], lse_s[fin], rtol=1e-4, atol=1e-3)
-    if oracle_too:
-        # selection by the band rule; then, in every unit whose selection is
-        # the oracle's own, the attention output of its heads against the oracle
-        ref = run.oracle_step()
-        check_selection(sel_f, nsel_f, ref["scores"], ref["sel"], ref["nsel"])
-        gs, gn = sel_f.cpu().numpy(), nsel_f.cpu().numpy()
-        G = run.d.Hq // run.d.Hkv
-        same = 0
-        for b in range(run.d.B):
-            for g in range(run.d.Hkv):
-                k = int(gn[b, g])
-                if not np.array_equal(gs[b, g, :k], ref["sel"][b, g, :k]):
-                    continue
-                same += 1
-                h = slice(g * G, (g + 1) * G)
-                assert_out_close(out_f[b, h], lse_f[b, h], ref["out"][b, h], ref["lse"][b, h],
-                                 f"one-call decode, unit ({b},{g})")
-        return same
-    return None
+    if not oracle_too:
+        return None
+    ref = run.oracle_step()
+    check_selection(sel_f, nsel_f, ref["scores"], ref["sel"], ref["nsel"])
+    exp_out, exp_lse, same = oracle_on_valid_choice(run.od, run.h, run.prefix, run.window,
+                                                     run.scale, sel_f, nsel_f, ref)
+    assert_out_close(out_f, lse_f, exp_out, exp_lse, "one-call decode")
+    G = run.d.Hq // run.d.Hkv
+    for b in range(run.d.B):
+        for g in range(run.d.Hkv):
+            h = slice(g * G, (g + 1) * G)
+            assert_out_close(out_f[b, h], lse_f[b, h], exp_out[b, h], exp_lse[b, h],
+                             f"one-call decode, unit ({b},{g})")
+    return same
 
 
 @pytest.mark.parametrize("w", [wl.TINY, wl.CTX32K, wl.CTX64K], ids=lambda w: w.name)
@@ -330,11 +328,34 @@ def test_one_call_edge_geometry(lens, P, W, budget, cuda):
     check_one_call(Run(wl.make_case(w, cuda)))
 
 
-def test_one_call_many_units_uses_separate_kernels(cuda):
-    """More than 32 (sequence, kv-head) units: the separate-kernel path."""
-    w = small(B=20, Hq=16, Hkv=2, lens=tuple(900 + 37 * i for i in range(20)), prefix=16,
-              window=64, budget=256)
-    check_one_call(Run(wl.make_case(w, cuda)), oracle_too=False)
+@pytest.mark.parametrize("G", [1, 8, 16])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_one_call_many_units(G, D, cuda):
+    """More than 32 (sequence, kv-head) units: the separate kernels (scoring,
+    selection, decode, combine) behind the one call, against the separate
+    calls and the oracle, every unit."""
+    w = small(B=20, Hq=2 * G, Hkv=2, D=D, lens=tuple(900 + 37 * i for i in range(20)),
+              prefix=16, window=64, budget=256)
+    check_one_call(Run(wl.make_case(w, cuda)))
+
+
+@pytest.mark.parametrize("lens,P,W,budget", [
+    ((0,) * 3 + (700,) * 30, 16, 16, 64),              # empty sequences
+    ((40,) * 17 + (1000,) * 16, 16, 32, 64),           # prefix + window cover some sequences
+    ((17,) * 11 + (300, 33) * 11, 5, 7, 32),           # candidates fewer than the cluster's CTAs
+    ((4096 + 5,) * 33, 64, 256, 512),                  # ragged tail page
+    (tuple(600 + 61 * i for i in range(33)), 0, 0, 16),  # no prefix or window, k = 1
+])
+def test_one_call_many_units_edge_geometry(lens, P, W, budget, cuda):
+    w = small(B=len(lens), Hq=4, Hkv=1, lens=lens, prefix=P, window=W, budget=budget)
+    check_one_call(Run(wl.make_case(w, cuda)))
+
+
+def test_one_call_many_units_ctx64k_batch8(cuda):
+    """Batch 8 x 8 kv-heads at 64k (64 units, D = 128), the benchmark's
+    larger-batch shape: every unit against the oracle."""
+    same = check_one_call(Run(wl.make_case(wl.CTX64K_B8, cuda)))
+    assert same >= 32
 
 
 @pytest.mark.parametrize("window", [0, 15, 16, 64])
