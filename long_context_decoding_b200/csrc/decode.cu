@@ -60,7 +60,7 @@ struct DecCfg {
     static __host__ __device__ size_t smem_bytes(int units) {
         return 1024 /* alignment slack */ + kStageArea + kMl + kItems + unit_bytes(units);
     }
-    // uoff [units + 1] | uinfo [units] (int2: validated seq_len, unused)
+    // uoff [units + 1] | uinfo [units] (int2: validated seq_len, fixed items of the pass)
     static __host__ __device__ size_t unit_bytes(int units) {
         return (((size_t)(units + 1) * 4 + 15) & ~(size_t)15) + (size_t)units * 8;
     }
@@ -204,20 +204,23 @@ decode_kernel(DecodeParams p) {
 
     // Phase 0 streams the fixed pages (prefix and window), which do not depend
     // on the selection; phase 1 the selected pages.  With p.early set, phase 0
-    // runs while the selection kernel ahead is still working.
-    for (int ph = 0; ph < 2; ++ph) {
-        if (ph == 1 && p.early) {
+    // runs while the selection kernel ahead is still working.  Without it
+    // both lists form one pass: each unit's fixed pages, then its selected
+    // pages, flattened and split together (one chain of round trips, not two).
+    const int passes = p.early ? 2 : 1;
+    for (int ph = 0; ph < passes; ++ph) {
+        if (ph == 1) {
             pdl_wait();         // the selection is complete and visible
             pdl_launch_dependents();
         }
+        const bool with_fixed = ph == 0, with_sel = ph == 1 || !p.early;
         __syncthreads();        // uinfo written; smem of the previous phase free
-        // ---- per-unit list lengths and their exclusive scan
+        // ---- per-unit list lengths (fixed in uinfo.y) and their exclusive scan
         for (int u = tid; u < units; u += C::kThreads) {
             const SeqGeom sg = seq_geom(uinfo[u].x, p.prefix, p.window);
+            const int nf = with_fixed ? fixed_list(sg, p.dense).total() : 0;
             int n = 0;
-            if (ph == 0) {
-                n = fixed_list(sg, p.dense).total();
-            } else if (!p.dense && sg.c_lo < sg.c_hi) {
+            if (with_sel && !p.dense && sg.c_lo < sg.c_hi) {
                 n = p.n_sel[u];
                 const int cap = p.s.max_sel < sg.c_hi - sg.c_lo ? p.s.max_sel : sg.c_hi - sg.c_lo;
                 if (n < 0 || n > cap) {
@@ -225,7 +228,8 @@ decode_kernel(DecodeParams p) {
                     n = n < 0 ? 0 : cap;
                 }
             }
-            uoff[u] = n;
+            uinfo[u].y = nf;
+            uoff[u] = nf + n;
         }
         __syncthreads();
         if (warp == 0) {
@@ -256,8 +260,10 @@ decode_kernel(DecodeParams p) {
         const long long s = blockIdx.x < (unsigned)n_cta ? T * blockIdx.x / n_cta : T;
         const long long e = blockIdx.x < (unsigned)n_cta ? T * (blockIdx.x + 1) / n_cta : T;
         if (blockIdx.x == 0) {   // units without pages in this phase: no records
-            for (int u = tid; u < units; u += C::kThreads)
+            for (int u = tid; u < units; u += C::kThreads) {
                 if (uoff[u + 1] == uoff[u]) rr2[2 * u + ph] = make_int2(0, -1);
+                if (passes == 1) rr2[2 * u + 1] = make_int2(0, -1);   // one pass: region 0 only
+            }
         }
         if (s >= e) continue;
 
@@ -269,13 +275,14 @@ decode_kernel(DecodeParams p) {
             const SeqGeom sg = seq_geom(uinfo[u].x, p.prefix, p.window);
             int page = 0, mask = kMaskAll;
             bool ok = true;
-            if (ph == 0) {
+            if (j < uinfo[u].y) {
                 fixed_item(sg, fixed_list(sg, p.dense), j, page, mask);
             } else {
+                const int js = j - uinfo[u].y;
                 const int32_t* su = p.sel + (size_t)u * p.s.max_sel;
-                page = su[j];
+                page = su[js];
                 mask = kMaskRest;
-                ok = page >= sg.c_lo && page < sg.c_hi && (j == 0 || su[j - 1] < page);
+                ok = page >= sg.c_lo && page < sg.c_hi && (js == 0 || su[js - 1] < page);
                 if (!ok) latch_flag(p.flags, CSA_DEVFLAG_BAD_SELECTION);
             }
             int phys = -1;

@@ -205,30 +205,44 @@ def test_chunk_append_prefill(cuda):
 
 
 def test_repeat_calls_reuse_workspace(cuda):
-    """Tickets left at zero: the same workspace serves many calls."""
+    """The same workspace serves many calls: repeated decodes are bit-identical
+    (the first, straight after the selection, streams its prefix/window pages
+    in a pass of their own and differs by rounding only), and all match the
+    oracle."""
     run = Run(wl.make_case(wl.TINY, cuda))
     run.gpu_meta()
     run.gpu_select()
-    out1, _ = run.gpu_decode(run.layer.sel, run.layer.n_sel)
-    for _ in range(5):
-        out2, _ = run.gpu_decode(run.layer.sel, run.layer.n_sel)
+    out1, lse1 = run.gpu_decode(run.layer.sel, run.layer.n_sel)
+    outs = [run.gpu_decode(run.layer.sel, run.layer.n_sel) for _ in range(5)]
     torch.cuda.synchronize()
-    assert torch.equal(out1, out2)
+    for o, l in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1])
+    ref = run.oracle_step()
+    assert_out_close(out1, lse1, ref["out"], ref["lse"], "decode after the selection")
+    assert_out_close(outs[0][0], outs[0][1], ref["out"], ref["lse"], "repeated decode")
 
 
 def test_fixed_pages_streamed_before_the_selection_ends(cuda):
     """Right after csa_score_select on the same stream, the decode streams the
-    prefix and window pages while the selection kernel still runs; the result
-    is bit-identical to a decode that waits for everything first."""
+    prefix and window pages while the selection kernel still runs (a pass of
+    their own); a decode that waits for everything first takes both lists in
+    one pass.  Both match the oracle; repeats of each are bit-identical."""
     run = Run(wl.make_case(wl.CTX32K, cuda))
     run.gpu_meta()
+    ref = run.oracle_step()
+    osel = torch.from_numpy(np.ascontiguousarray(ref["sel"])).to(cuda)
+    onsel = torch.from_numpy(ref["nsel"]).to(cuda)
+    prev = None
     for _ in range(3):
         run.gpu_select(scores=False)
-        out_e, lse_e = run.gpu_decode(run.layer.sel, run.layer.n_sel)   # overlapped
-        out_w, lse_w = run.gpu_decode(run.layer.sel, run.layer.n_sel)   # waits first
+        out_e, lse_e = run.gpu_decode(osel, onsel)   # overlapped with the selection
+        out_w, lse_w = run.gpu_decode(osel, onsel)   # waits first
         torch.cuda.synchronize()
-        assert torch.equal(out_e, out_w)
-        assert torch.equal(lse_e, lse_w)
+        assert_out_close(out_e, lse_e, ref["out"], ref["lse"], "early decode")
+        assert_out_close(out_w, lse_w, ref["out"], ref["lse"], "waiting decode")
+        if prev is not None:
+            assert torch.equal(out_e, prev[0]) and torch.equal(out_w, prev[1])
+        prev = (out_e, out_w)
     assert csa.device_status(run.ws) == 0
 
 
