@@ -65,6 +65,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=0,
                     help="use only the first N layers (small cases for ncu captures)")
+    ap.add_argument("--layer-cfg", type=int, default=-1,
+                    help="with --layers, start the stack's (window, budget) cycle at pair i "
+                         "(e.g. --layers 1 --layer-cfg 3: one layer with the largest pair)")
     ap.add_argument("--no-fp8", action="store_true", help="skip the fp8-metadata line")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the compact sparse-vs-dense sweep of the default run")
@@ -858,6 +861,9 @@ def main():
     base = wl.CTX256K if args.workload == "ctx256k" else replace(wl.CTX64K, steps=0)
     if args.layers:
         base = replace(base, layers=args.layers)
+    if args.layer_cfg >= 0 and base.layer_cfgs:
+        i = args.layer_cfg % len(base.layer_cfgs)
+        base = replace(base, layer_cfgs=base.layer_cfgs[i:] + base.layer_cfgs[:i])
     try:
         if args.impl == "reference":
             run_reference(args, dist, base)

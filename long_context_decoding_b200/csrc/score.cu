@@ -67,6 +67,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
     return h2;
 }
 
+// 2^e as a normal float, e clamped to [-126, 127] (built from its exponent bits).
+__device__ __forceinline__ float pow2_normal(int e) {
+    e = e < -126 ? -126 : (e > 127 ? 127 : e);
+    return __int_as_float((e + 127) << 23);
+}
+// x * 2^e, exact while the result stays in the normal range, for e in
+// [-252, 254] (two power-of-two factors, each a normal float).
+__device__ __forceinline__ float scale_pow2(float x, int e) {
+    const int e1 = e / 2;
+    return x * pow2_normal(e1) * pow2_normal(e - e1);
+}
+
 // 16-byte load that does not allocate in L1 (the metadata is read once).
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     uint4 v;
@@ -396,9 +408,10 @@ struct RingCfg {
 // component within 2^-31 of the head's largest (the rest, which move the sum
 // by less than its fp32 rounding, round to the f16 grid), and never
 // saturated, whatever the magnitude of q.  The row's sums are scaled back by
-// 2^(e + f), exactly.
+// 2^(e + f), exactly (two power-of-two factors: exact for |e + f| up to
+// about 250, which covers every exponent bf16 keys and queries produce).
 template <int D, int NB, bool F8>
-__global__ void __launch_bounds__(RingCfg<D, F8>::kThreads, 2)
+__global__ void __launch_bounds__(RingCfg<D, F8>::kThreads, (F8 && D <= 128) ? 4 : 2)
 score_ring_kernel(ScoreParams p) {
     using C = RingCfg<D, F8>;
     extern __shared__ __align__(16) int smem_i[];
@@ -495,7 +508,7 @@ score_ring_kernel(ScoreParams p) {
                             uint32_t r;
                             asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;"
                                 : "=r"(r)
-                                : "f"(ldexpf(bf16_hi(w), -f)), "f"(ldexpf(bf16_lo(w), -f)));
+                                : "f"(scale_pow2(bf16_hi(w), -f)), "f"(scale_pow2(bf16_lo(w), -f)));
                             qf[kk][nb][h] = r;
                         }
                     // accumulator columns 2t and 2t + 1 belong to the heads
@@ -547,10 +560,10 @@ score_ring_kernel(ScoreParams p) {
             const int e8 = *reinterpret_cast<const int*>(rows + (gq + 8) * C::kStride + 2 * D);
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-                acc[nb][0] = ldexpf(acc[nb][0] + acc2[nb][0], e0 + qexp[nb][0]);
-                acc[nb][1] = ldexpf(acc[nb][1] + acc2[nb][1], e0 + qexp[nb][1]);
-                acc[nb][2] = ldexpf(acc[nb][2] + acc2[nb][2], e8 + qexp[nb][0]);
-                acc[nb][3] = ldexpf(acc[nb][3] + acc2[nb][3], e8 + qexp[nb][1]);
+                acc[nb][0] = scale_pow2(acc[nb][0] + acc2[nb][0], e0 + qexp[nb][0]);
+                acc[nb][1] = scale_pow2(acc[nb][1] + acc2[nb][1], e0 + qexp[nb][1]);
+                acc[nb][2] = scale_pow2(acc[nb][2] + acc2[nb][2], e8 + qexp[nb][0]);
+                acc[nb][3] = scale_pow2(acc[nb][3] + acc2[nb][3], e8 + qexp[nb][1]);
             }
         }
         int p0, p8;
