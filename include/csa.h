@@ -56,16 +56,20 @@
  *    may start while the previous kernel on the stream finishes.  Each call
  *    waits for the preceding work before it reads anything, with two
  *    exceptions.  (1) csa_meta_update, csa_score_select and
- *    csa_sparse_attention read `page_table` and `seq_lens` early: those two
- *    must not come from the kernel launched just before the call if that
- *    kernel releases its dependents early (a host copy, an event, a plain
- *    kernel or a call of this library is fine).  (2) When the
- *    previous call of this library on the same stream was csa_score_select,
- *    csa_decode / csa_decode_full stream the prefix and window pages while
- *    the selection kernel is still running: their `q`, `k_cache`,
- *    `v_cache`, `page_table` and `seq_lens` must not be written between the
- *    two calls.  The library remembers the last call per stream handle on
- *    the host; this is its only state outside the workspace.
+ *    csa_sparse_attention read `page_table` and `seq_lens` early, and
+ *    csa_decode / csa_decode_full read `page_table`, `seq_lens`, `sel_pages`
+ *    and `n_sel` early (the dependency wait comes before the cache and the
+ *    workspace): those inputs must not come from the kernel launched just
+ *    before the call if that kernel releases its dependents early (a host
+ *    copy, an event, a plain kernel or a call of this library is fine; the
+ *    selections of csa_score_select and csa_select_scores count, see (2)).
+ *    (2) When the previous call of this library on the same stream was
+ *    csa_score_select or csa_select_scores, csa_decode / csa_decode_full
+ *    stream the prefix and window pages while the selection kernel is still
+ *    running and read the selection only after their wait: their `q`,
+ *    `k_cache`, `v_cache`, `page_table` and `seq_lens` must not be written
+ *    between the two calls.  The library remembers the last call per stream
+ *    handle on the host; this is its only state outside the workspace.
  *  - Page ids that fall outside [0, num_pages), selected pages outside the
  *    candidate range, and a selection that is not strictly ascending are
  *    detected on the device: the page is skipped and a flag is latched in

@@ -531,7 +531,11 @@ int csa_select_scores(const csa_dims* d, const float* scores, const int32_t* seq
     lp.flags = at<uint32_t>(workspace, w.flags);
     lp.smem_keys = 0;
     lp.s = s;
-    return launch_status(launch_select(lp, st));
+    rc = launch_status(launch_select(lp, st));
+    // the selection kernel lets the next grid start before it writes sel: a
+    // decode that follows reads the selection only after its wait
+    note_stream_call(stream, rc == CSA_OK ? kCallScoreSelect : kCallOther);
+    return rc;
 }
 
 int csa_shard_selection(const csa_dims* d, const int32_t* sel_pages, const int32_t* n_sel,

@@ -177,10 +177,9 @@ decode_kernel(DecodeParams p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int Hkv = p.s.Hkv, G = p.s.G, Hq = p.s.Hq;
     int2* rr2 = reinterpret_cast<int2*>(p.rec_range);   // [unit][phase]: first, last CTA
-    if (!p.early) {   // wait for everything ahead before reading anything
-        pdl_wait();
-        pdl_launch_dependents();
-    }
+    // Until the dependency wait the kernel reads only caller inputs (lengths,
+    // selection, page table); the cache, the record ranges and the partial
+    // records, which the kernels ahead may still use, only after it.
     for (int u = tid; u < units; u += C::kThreads) {
         int L = p.seq_lens[u / Hkv];
         if (L < 0 || L > p.s.MP * kPage) {
@@ -259,13 +258,6 @@ decode_kernel(DecodeParams p) {
         const int n_cta = (int)(want < (long long)gridDim.x ? want : gridDim.x);
         const long long s = blockIdx.x < (unsigned)n_cta ? T * blockIdx.x / n_cta : T;
         const long long e = blockIdx.x < (unsigned)n_cta ? T * (blockIdx.x + 1) / n_cta : T;
-        if (blockIdx.x == 0) {   // units without pages in this phase: no records
-            for (int u = tid; u < units; u += C::kThreads) {
-                if (uoff[u + 1] == uoff[u]) rr2[2 * u + ph] = make_int2(0, -1);
-                if (passes == 1) rr2[2 * u + 1] = make_int2(0, -1);   // one pass: region 0 only
-            }
-        }
-        if (s >= e) continue;
 
         // ---- resolve the physical page of every item of this CTA's slice
         for (long long x = s + tid; x < e; x += C::kThreads) {
@@ -296,6 +288,17 @@ decode_kernel(DecodeParams p) {
             items[x - s] = make_int2(phys, page * 4 + mask);
         }
         __syncthreads();
+        if (!p.early) {          // the one pass: wait for everything ahead now
+            pdl_wait();
+            pdl_launch_dependents();
+        }
+        if (blockIdx.x == 0) {   // units without pages in this phase: no records
+            for (int u = tid; u < units; u += C::kThreads) {
+                if (uoff[u + 1] == uoff[u]) rr2[2 * u + ph] = make_int2(0, -1);
+                if (passes == 1) rr2[2 * u + 1] = make_int2(0, -1);   // one pass: region 0 only
+            }
+        }
+        if (s >= e) continue;
 
         const int u_first = find_unit(uoff, units, s);
         const int u_last = find_unit(uoff, units, e - 1);

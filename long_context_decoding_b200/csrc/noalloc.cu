@@ -116,7 +116,11 @@ extern "C" int csa_decode_noalloc(const csa_dims* d, const void* q, const void* 
     p.rec_range = reinterpret_cast<int4*>(scratch + ranges_off);
     p.partials = reinterpret_cast<float*>(scratch + partials_off);
     p.phase_floats = slots * decode_record_floats(s);
-    p.early = 0;                 // the scratch is shared: wait before touching it
+    // as csa_decode: right after a selection call on this stream, the prefix
+    // and window pages stream before the dependency wait and the selection is
+    // read after it; otherwise the caller inputs are read before the wait and
+    // the scratch is touched only after it
+    p.early = last_stream_call(stream) == kCallScoreSelect ? 1 : 0;
     p.s = s;
     note_stream_call(stream, kCallOther);
     if (launch_decode(p, st) != cudaSuccess) {
