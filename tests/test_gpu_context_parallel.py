@@ -14,7 +14,7 @@ import oracle
 from long_context_decoding_b200 import context_parallel as cp
 from long_context_decoding_b200 import csa
 from long_context_decoding_b200 import workloads as wl
-from parity import PS, Run, assert_out_close, check_selection
+from parity import PS, Run, assert_out_close, check_selection, oracle_on_valid_choice
 from test_context_parallel import ListExchange, lse_merge
 
 pytestmark = pytest.mark.gpu
@@ -94,6 +94,41 @@ def test_select_scores_equals_score_select(w, cuda):
         for h in range(run.d.Hkv):
             k = int(n2[b, h])
             assert torch.equal(sel2[b, h, :k], lay.sel[b, h, :k])
+
+
+@pytest.mark.parametrize("noalloc", [False, True], ids=["decode", "decode_noalloc"])
+def test_decode_straight_after_select_scores(noalloc, cuda):
+    """csa_decode (and csa_decode_noalloc) issued straight after
+    csa_select_scores on the same stream, no host sync in between: the
+    selection kernel lets the next grid start before it writes the selection,
+    so the decode must read it only after its dependency wait.  Repeated, the
+    outputs match the oracle's attention over the (band-valid) selection."""
+    run = Run(wl.make_case(wl.CTX32K, cuda))
+    run.gpu_meta()
+    sc = torch.full((run.d.B, run.d.Hkv, run.d.max_pages_per_seq), float("nan"), device=cuda)
+    lay = run.layer
+    csa.score_select(run.d, run.c.q, lay.meta, run.c.page_table, run.c.seq_lens, run.prefix,
+                     run.window, run.budget, lay.sel, lay.n_sel, run.ws, scores_out=sc)
+    ref = run.oracle_step()
+    for _ in range(3):
+        sel2 = torch.full_like(lay.sel, -5)
+        n2 = torch.full_like(lay.n_sel, -5)
+        out = torch.empty((run.d.B, run.d.Hq, run.d.D), dtype=torch.bfloat16, device=cuda)
+        lse = torch.empty((run.d.B, run.d.Hq), dtype=torch.float32, device=cuda)
+        csa.select_scores(run.d, sc, run.c.seq_lens, run.prefix, run.window, run.budget, sel2,
+                          n2, run.ws)
+        if noalloc:
+            csa.decode_noalloc(run.d, run.c.q, run.c.k_cache, run.c.v_cache, run.c.page_table,
+                               run.c.seq_lens, sel2, n2, run.prefix, run.window, out, lse)
+        else:
+            csa.decode(run.d, run.c.q, run.c.k_cache, run.c.v_cache, run.c.page_table,
+                       run.c.seq_lens, sel2, n2, run.prefix, run.window, out, run.ws, lse)
+        torch.cuda.synchronize()
+        assert csa.device_status(run.ws) == 0
+        check_selection(sel2, n2, ref["scores"], ref["sel"], ref["nsel"])
+        exp_out, exp_lse, _ = oracle_on_valid_choice(run.od, run.h, run.prefix, run.window,
+                                                     run.scale, sel2, n2, ref)
+        assert_out_close(out, lse, exp_out, exp_lse, "decode after csa_select_scores")
 
 
 def emulate(run: Run, R: int):

@@ -46,6 +46,10 @@ def full_check(run: Run, dense=True):
         osel = pad
     out, lse = run.gpu_decode(osel, onsel)
     errs = {"sparse": assert_out_close(out, lse, ref["out"], ref["lse"], "sparse decode")}
+    # again, not right after a selection: both lists in one pass
+    out1, lse1 = run.gpu_decode(osel, onsel)
+    errs["sparse_one_pass"] = assert_out_close(out1, lse1, ref["out"], ref["lse"],
+                                               "sparse decode, one pass")
     assert csa.device_status(run.ws) == 0
     if dense:
         dout, dlse = run.gpu_dense()
