@@ -490,7 +490,7 @@ def run_ours(args, dist: Dist, base: wl.Workload):
             "kernel": "score_direct_kernel (Quest scoring; the largest share of the launch list)",
             "kernel_achieved": ach, "kernel_frac": ach / peak, "kernel_traffic": traffic,
             "kernel_traffic_source": (f"ncu dram__bytes_read+write per launch, {traffic_src}, "
-                                      "profiles/score_kernel_ctx256k_layer.md")
+                                      "profiles/traffic_layer_step_ctx256k.md")
                                      if traffic else None,
             "kernel_note": "metadata bytes of the candidate pages (|C| x 4D per unit) / "
                            "CUDA-event time per call, from graph replays of budget-0 "
