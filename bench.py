@@ -69,6 +69,9 @@ def parse_args():
                     help="with --layers, start the stack's (window, budget) cycle at pair i "
                          "(e.g. --layers 1 --layer-cfg 3: one layer with the largest pair)")
     ap.add_argument("--no-fp8", action="store_true", help="skip the fp8-metadata line")
+    ap.add_argument("--fp8-step", action="store_true",
+                    help="with --profile: the timed steps score from the fp8 metadata copy "
+                         "(csa_meta_update_fp8 + csa_sparse_attention_fp8), for ncu captures")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the compact sparse-vs-dense sweep of the default run")
     ap.add_argument("--sweep", action="store_true",
@@ -384,12 +387,22 @@ def run_ours(args, dist: Dist, base: wl.Workload):
     st = Stack(rank_workload(base, dist.rank, K + W), dev)
     w = st.w
     nl = len(st.layers)
+    what = "all"
+    if args.fp8_step:
+        if not args.profile:
+            raise SystemExit("bench.py: --fp8-step is a profiling mode (use it with --profile)")
+        for lay in st.layers:
+            lay.meta8 = st.csa.new_meta8(st.d, st.dev)
+            st.csa.meta_update_fp8(st.d, lay.k_cache, lay.v_cache, lay.meta, lay.meta8,
+                                   lay.page_table, st.lens[0], None, None,
+                                   st.d.max_pages_per_seq * 16, st.ws)
+        what = "all_fp8"
     # eager pass over every step: sets kernel attributes, checks the flags
     for s in range(K + W):
-        st.calls(s)
+        st.calls(s, what=what)
     torch.cuda.synchronize()
     assert st.csa.device_status(st.ws) == 0, "device flag after the eager pass"
-    graphs = [st.graph(lambda s=s: st.calls(s)) for s in range(K + W)]
+    graphs = [st.graph(lambda s=s: st.calls(s, what=what)) for s in range(K + W)]
     for s in range(W):
         graphs[s].replay()
     clocks = None if args.profile else Clocks(dev)
@@ -510,6 +523,7 @@ def run_ours(args, dist: Dist, base: wl.Workload):
         # ---- 64k single layer (the other context of the metric)
         if not args.no_secondary and base.name == wl.CTX256K.name:
             line["ctx64k"] = secondary_64k(dev, dist)
+            line["many_units"] = secondary_many_units(dev, dist, line)
 
         # ---- sparse against dense over context length, and the cost model
         if not args.no_sweep and base.name == wl.CTX256K.name:
@@ -681,6 +695,47 @@ def secondary_64k(dev, dist: Dist):
             "dense_us": 1e6 * tdn, "dense_gbs": by["dense"] / tdn / 1e9,
             "speedup_vs_dense": tdn / t,
             "timing": "batches of 20 graph replays, each after a 256 MB L2 flush (read); the flush time subtracted; median of 3 batches"}
+
+
+def secondary_many_units(dev, dist: Dist, line):
+    """One layer step of the 64k decode at batch 8 x 8 kv-heads (64
+    (sequence, kv-head) units, D = 128): one csa_sparse_attention call,
+    which beyond 32 units runs as scoring, selection, decode and combine
+    launches.  Timed like the 64k line (L2 read-flush before every replay);
+    its per-byte rate is set against the 8-unit 64k layer and the 256k
+    stack's layer step."""
+    from long_context_decoding_b200 import csa
+    w = wl.CTX64K_B8
+    c = wl.make_case(w, dev)
+    d = csa.make_dims(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.num_pages, w.max_sel)
+    lay = csa.Layer(d, c.k_cache, c.v_cache, c.page_table, c.seq_lens, w.prefix, w.window,
+                    w.budget)
+    lay.rebuild_meta()
+    scrub = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MB
+    sink = torch.zeros((), device=dev)
+
+    def flush():
+        torch.sum(scrub, dim=0, out=sink)
+
+    t = dist.max(graph_time(lambda: lay.step(c.q, fused=True), 20, 5, flush))
+    flags = csa.device_status(lay.ws)
+    by = cost.layer_bytes(w.seq_lens, w.Hq, w.Hkv, w.D, w.prefix, w.window, w.budget)
+    peak, _ = hbm_peak()
+    ach = by["sparse"] / t / 1e9
+    ref64 = line.get("ctx64k", {}).get("achieved_gbs")
+    ref256 = line.get("layer_step", {}).get("achieved_gbs")
+    del lay, c
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "units": w.B * w.Hkv, "value": dist.world * w.B / t,
+            "unit": UNIT, "us_per_layer_step": 1e6 * t, "algorithmic_bytes": by["sparse"],
+            "achieved_gbs": ach, "frac_of_measured_peak": ach / peak,
+            "rate_vs_ctx64k": ach / ref64 if ref64 else None,
+            "rate_vs_256k_layer_step": ach / ref256 if ref256 else None,
+            "device_flags": flags,
+            "path": "more than 32 units: scoring, cluster selection, decode (prefix/window "
+                    "pages during the selection) and combine as separate launches",
+            "timing": "batches of 20 graph replays, each after a 256 MB L2 flush (read); the "
+                      "flush time subtracted; median of 3 batches"}
 
 
 def planted_recall(sel, nsel, planted):

@@ -16,7 +16,7 @@
 // Data path.  The kernels stream one metadata row per candidate (page,
 // kv-head) from random physical pages and do ~2 flop per byte: they are
 // bound by memory, and on B200 the rate of random row requests (~12 G rows/s
-// for rows of 256 to 512 bytes) matters as much as the bytes.  Two load
+// for rows of 256 to 512 bytes) matters as much as the bytes.  Three load
 // paths, chosen per shape by measurement:
 //   * direct (bf16 metadata, D <= 128): every warp loads its own tiles
 //     straight into the registers that feed the MMA.  With the k index of the
@@ -24,13 +24,18 @@
 //     needs exactly the 16-byte chunks t, t+4, ... of rows g and g+8, so a
 //     tile is 2D/16 plain 16-byte loads per lane, with no staging and no
 //     barriers.
-//   * ring (bf16 metadata at D = 256, and the fp8 copy): each warp copies
-//     whole rows of its tiles into a private shared-memory ring with 16-byte
-//     cp.async (one 512-byte row per instruction), keeps several tiles in
-//     flight, and reads a landed tile into MMA fragments with ldmatrix.
-// Both: the candidates of all (sequence, kv-head) units are flattened and
-// split evenly over the grid; each CTA copies its slice of the page table
-// into shared memory once, before the dependency wait.  A TMA bulk copy per
+//   * ring (bf16 metadata at D = 256, and the fp8 copy of other shapes):
+//     each warp copies whole rows of its tiles into a private shared-memory
+//     ring with 16-byte cp.async (one 512-byte row per instruction), keeps
+//     several tiles in flight, and reads a landed tile into MMA fragments
+//     with ldmatrix.
+//   * page-major (the fp8 copy at 4 or 8 kv-heads): the CTA copies whole
+//     pages, all kv-heads' rows of a page as one contiguous run, into a
+//     shared ring; warp g scores kv-head g.
+// All: the candidates of all (sequence, kv-head) units -- of all sequences,
+// for the page-major path -- are flattened and split evenly over the grid;
+// each CTA copies its slice of the page table into shared memory once,
+// before the dependency wait.  A TMA bulk copy per
 // row (512 bytes) is limited by its per-copy issue cost to ~30% of the copy
 // peak on B200, so neither path uses one.
 #include "common.cuh"
@@ -139,22 +144,26 @@ struct TileWalker {
     }
 };
 
-// Shared memory common to both kernels: page-table slice | 3 x [B + 1] ints.
-__host__ __device__ __forceinline__ size_t score_common_bytes(int B) {
-    return (size_t)kScorePtCap * 4 + 12 * (size_t)(B + 1);
+// Shared memory common to the kernels: page-table slice (cap entries) |
+// 3 x [B + 1] ints.
+__host__ __device__ __forceinline__ size_t score_common_bytes(int B, int cap = kScorePtCap) {
+    return (size_t)cap * 4 + 12 * (size_t)(B + 1);
 }
 
-// The prologue of both kernels: candidates per sequence, their exclusive scan
-// over (sequence, kv-head), this CTA's range [s, e) of the flattened list and
-// its page-table slice -- all from caller inputs, before the dependency wait
-// -- then the wait (the metadata was written by the previous kernel on the
-// stream).  Returns the walker template (range not started).
+// The prologue of the kernels: candidates per sequence, their exclusive scan
+// over (sequence, kv-head) -- or over sequences alone when Hkv is passed as 1
+// (the page-major kernel, whose items are pages) -- this CTA's range [s, e)
+// of the flattened list and its page-table slice (at most cap entries, which
+// the grid guarantees) -- all from caller inputs,
+// before the dependency wait -- then the wait (the metadata was written by
+// the previous kernel on the stream).  Returns the walker template (range not
+// started).
 __device__ __forceinline__ TileWalker score_setup(const ScoreParams& p, int* smem_i, int& s,
-                                                  int& e) {
-    const int B = p.s.B, Hkv = p.s.Hkv, MP = p.s.MP;
+                                                  int& e, int Hkv, int cap = kScorePtCap) {
+    const int B = p.s.B, MP = p.s.MP;
     const int tid = threadIdx.x, lane = tid & 31, nthr = blockDim.x;
     int* pt = smem_i;
-    int* seq_n = pt + kScorePtCap;
+    int* seq_n = pt + cap;
     int* seq_clo = seq_n + (B + 1);
     int* seq_off = seq_clo + (B + 1);
     for (int b = tid; b < B; b += nthr) {
@@ -299,7 +308,7 @@ score_direct_kernel(ScoreParams p) {
     using C = DirectCfg<D, NB>;
     extern __shared__ __align__(16) int smem_i[];
     int s, e;
-    TileWalker walk = score_setup(p, smem_i, s, e);
+    TileWalker walk = score_setup(p, smem_i, s, e, p.s.Hkv);
     if (s >= e) return;
     const int* pt = smem_i;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -368,6 +377,66 @@ score_direct_kernel(ScoreParams p) {
     kr.flush(p, lane);
 }
 
+// B fragments of [q- | q+] for unit (b, g): MMA kk covers the 16 channels
+// [16 kk, 16 kk + 16) of the [min | max] row (min pairs with q-).  F8: each
+// head's q scaled by 2^-f and converted to f16 (see score_ring_kernel), with
+// qexp[nb] = the exponents f of the heads of accumulator columns 2t, 2t + 1.
+template <int D, int NB, bool F8>
+__device__ __forceinline__ void load_q_frags(const ScoreParams& p, int b, int g, int lane,
+                                             uint32_t (&qf)[D / 8][NB][2], int (&qexp)[NB][2]) {
+    const int gq = lane >> 2, tq = lane & 3, G = p.s.G;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        const int head = nb * 8 + gq;
+        const uint32_t* qw = reinterpret_cast<const uint32_t*>(
+            p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
+#pragma unroll
+        for (int kk = 0; kk < D / 8; ++kk) {
+            const bool is_max = 16 * kk >= D;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                // channel pair of k slots (2t, 2t+1) [h = 0] or (2t+8, 2t+9) [h = 1]
+                const int ch = F8 ? 16 * kk + 4 * tq + 2 * h : 16 * kk + 8 * h + 2 * tq;
+                const int qc = is_max ? ch - D : ch;
+                const uint32_t v = head < G ? __ldg(qw + qc / 2) : 0u;
+                qf[kk][nb][h] = is_max ? pos_part(v) : neg_part(v);
+            }
+        }
+    }
+    if constexpr (F8) {
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            // largest |q| of head nb * 8 + g: this lane holds a quarter
+            // of its channels (each once in the q- and once in the q+ half)
+            float amax = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < D / 8; ++kk)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(qf[kk][nb][h])),
+                                             fabsf(bf16_hi(qf[kk][nb][h]))));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            const int f = amax > 0.f ? ilogbf(amax) - 14 : 0;
+#pragma unroll
+            for (int kk = 0; kk < D / 8; ++kk)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t w = qf[kk][nb][h];
+                    uint32_t r;
+                    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;"
+                        : "=r"(r)
+                        : "f"(scale_pow2(bf16_hi(w), -f)), "f"(scale_pow2(bf16_lo(w), -f)));
+                    qf[kk][nb][h] = r;
+                }
+            // accumulator columns 2t and 2t + 1 belong to the heads
+            // loaded by the lanes with g = 2t and g = 2t + 1
+            qexp[nb][0] = __shfl_sync(0xffffffffu, f, 8 * tq);
+            qexp[nb][1] = __shfl_sync(0xffffffffu, f, 8 * tq + 4);
+        }
+    }
+}
+
 // ------------------------------------------------------------ ring path
 // Shared-memory rings, one per warp, of kStages tiles of 16 rows; each warp
 // takes a contiguous 1/kWarps of the CTA's range.
@@ -416,12 +485,12 @@ score_ring_kernel(ScoreParams p) {
     using C = RingCfg<D, F8>;
     extern __shared__ __align__(16) int smem_i[];
     int s, e;
-    TileWalker walk = score_setup(p, smem_i, s, e);
+    TileWalker walk = score_setup(p, smem_i, s, e, p.s.Hkv);
     if (s >= e) return;
     const int* pt = smem_i;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int B = p.s.B, Hkv = p.s.Hkv, G = p.s.G;
-    const int gq = lane >> 2, tq = lane & 3;
+    const int B = p.s.B, Hkv = p.s.Hkv;
+    const int gq = lane >> 2;
     uint8_t* ring = reinterpret_cast<uint8_t*>(smem_i) + C::ring_offset(B) +
                     (size_t)warp * C::kStages * C::kTileSmem;
     int4* desc = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(smem_i) + C::desc_offset(B)) +
@@ -467,56 +536,7 @@ score_ring_kernel(ScoreParams p) {
         const int b = t.unit / Hkv, g = t.unit % Hkv;
         if (t.unit != cur_unit) {
             cur_unit = t.unit;
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const int head = nb * 8 + gq;
-                const uint32_t* qw = reinterpret_cast<const uint32_t*>(
-                    p.q + ((size_t)b * p.s.Hq + (size_t)g * G + (head < G ? head : 0)) * D);
-#pragma unroll
-                for (int kk = 0; kk < D / 8; ++kk) {
-                    const bool is_max = 16 * kk >= D;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        // channel pair of k slots (2t, 2t+1) [h = 0] or (2t+8, 2t+9) [h = 1]
-                        const int ch = F8 ? 16 * kk + 4 * tq + 2 * h : 16 * kk + 8 * h + 2 * tq;
-                        const int qc = is_max ? ch - D : ch;
-                        const uint32_t v = head < G ? __ldg(qw + qc / 2) : 0u;
-                        qf[kk][nb][h] = is_max ? pos_part(v) : neg_part(v);
-                    }
-                }
-            }
-            if constexpr (F8) {
-#pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    // largest |q| of head nb * 8 + g: this lane holds a quarter
-                    // of its channels (each once in the q- and once in the q+ half)
-                    float amax = 0.f;
-#pragma unroll
-                    for (int kk = 0; kk < D / 8; ++kk)
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(qf[kk][nb][h])),
-                                                     fabsf(bf16_hi(qf[kk][nb][h]))));
-                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                    const int f = amax > 0.f ? ilogbf(amax) - 14 : 0;
-#pragma unroll
-                    for (int kk = 0; kk < D / 8; ++kk)
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint32_t w = qf[kk][nb][h];
-                            uint32_t r;
-                            asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;"
-                                : "=r"(r)
-                                : "f"(scale_pow2(bf16_hi(w), -f)), "f"(scale_pow2(bf16_lo(w), -f)));
-                            qf[kk][nb][h] = r;
-                        }
-                    // accumulator columns 2t and 2t + 1 belong to the heads
-                    // loaded by the lanes with g = 2t and g = 2t + 1
-                    qexp[nb][0] = __shfl_sync(0xffffffffu, f, 8 * tq);
-                    qexp[nb][1] = __shfl_sync(0xffffffffu, f, 8 * tq + 4);
-                }
-            }
+            load_q_frags<D, NB, F8>(p, b, g, lane, qf, qexp);
         }
         const uint32_t tile = ring_s + (uint32_t)(stage * C::kTileSmem) + lm_off;
         // two accumulator chains (even and odd MMAs), summed at the end
@@ -606,6 +626,181 @@ score_ring_kernel(ScoreParams p) {
     kr.flush(p, lane);
 }
 
+// ------------------------------------------------------------ page-major fp8 path
+// The fp8 rows of all kv-heads of a page lie side by side (Hkv x (2D + 16)
+// bytes), so the CTA copies whole pages: one contiguous run per page instead
+// of Hkv separate rows, which raises the rate of random requests for these
+// short rows.  A CTA of HKV warps takes a range of the candidate pages of all
+// sequences (flattened over sequences); each stage of its shared ring holds
+// up to 16 consecutive candidate pages of one sequence, all kv-heads, copied
+// by every thread, and warp g scores the 16 x 2D tile of kv-head g with its
+// own q fragments (the same MMAs, operand order and scaling as the ring
+// kernel, so the scores agree with it bit for bit).  One CTA barrier per
+// stage.
+template <int D, int NB, int HKV>
+struct PmCfg {
+    static constexpr int kRowBytes = 2 * D + 16;             // one (page, kv-head) row
+    static constexpr int kRowChunks = kRowBytes / 16;
+    static constexpr int kPageChunks = HKV * kRowChunks;     // one page, every kv-head
+    static constexpr int kTileSmem = 16 * kRowBytes;         // kv-head g's rows of a stage
+    static constexpr int kStageSmem = HKV * kTileSmem;
+    static constexpr int kWarps = HKV;
+    static constexpr int kThreads = 32 * kWarps;
+    static constexpr int kPageIters = (kPageChunks + 31) / 32;   // per lane and page
+    // CTAs per SM: at 4 kv-heads and D <= 128, four (three stages each;
+    // measured faster than two or three CTAs with deeper rings), three where
+    // four would spill registers (16-head groups at D = 128); else two
+    static constexpr int kCtasPerSm =
+        (HKV == 4 && D <= 128) ? ((NB == 1 || D == 64) ? 4 : 3) : 2;
+    static constexpr int kRingBudget = (kCtasPerSm == 4 ? 52 : 70) * 1024;   // per CTA
+    static constexpr int kStagesFit = kRingBudget / kStageSmem;
+    static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
+    static_assert(kRowChunks % 2 == 1, "odd row stride: conflict-free ldmatrix");
+    // page-table slice: a CTA's share of the candidate pages, at most
+    // ceil(B * MP / grid) (the grid keeps it within kScorePtCap)
+    static __host__ __device__ int pt_cap(int B, int MP, int grid) {
+        const long long c = ((long long)B * MP + grid - 1) / grid;
+        return (int)((c + 3) & ~3ll);
+    }
+    static __host__ __device__ size_t desc_offset(int B, int cap) {
+        return (score_common_bytes(B, cap) + 15) & ~(size_t)15;
+    }
+    static __host__ __device__ size_t ring_offset(int B, int cap) {
+        return (desc_offset(B, cap) + (size_t)kStages * 16 + 127) & ~(size_t)127;
+    }
+    static __host__ __device__ size_t smem_bytes(int B, int cap) {
+        return ring_offset(B, cap) + (size_t)kStages * kStageSmem;
+    }
+};
+
+template <int D, int NB, int HKV>
+__global__ void __launch_bounds__(PmCfg<D, NB, HKV>::kThreads, PmCfg<D, NB, HKV>::kCtasPerSm)
+    score_pm_kernel(ScoreParams p) {
+    using C = PmCfg<D, NB, HKV>;
+    static_assert(C::kStages >= 2, "two stages at least");
+    extern __shared__ __align__(16) int smem_i[];
+    const int cap = C::pt_cap(p.s.B, p.s.MP, (int)gridDim.x);
+    int s, e;
+    TileWalker walk = score_setup(p, smem_i, s, e, 1, cap);   // items: candidate pages
+    if (s >= e) return;
+    const int* pt = smem_i;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gq = lane >> 2;
+    uint8_t* ring = reinterpret_cast<uint8_t*>(smem_i) + C::ring_offset(p.s.B, cap);
+    int4* desc = reinterpret_cast<int4*>(reinterpret_cast<uint8_t*>(smem_i) +
+                                         C::desc_offset(p.s.B, cap));
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    const uint32_t lm_off = (uint32_t)(((lane & 7) + 8 * ((lane >> 3) & 1)) * C::kRowBytes +
+                                       16 * (lane >> 4));
+
+    // copies of a stage: warp w copies pages w, w + HKV, ... of the group,
+    // lane l the 16-byte chunks l, l + 32, ... of a page's HKV rows, whose
+    // places in the stage (row g of tile g's page slot) are the same for
+    // every page; slots past the group and bad page ids are zero-filled
+    // (their scores are dropped)
+    uint32_t doff[C::kPageIters];
+#pragma unroll
+    for (int i = 0; i < C::kPageIters; ++i) {
+        const int j = lane + 32 * i, g = j / C::kRowChunks;
+        doff[i] = (uint32_t)(g * C::kTileSmem + 16 * (j - g * C::kRowChunks));
+    }
+    auto issue = [&](const TileInfo& t, int x0, int stage) {
+        const uint32_t dst = ring_s + (uint32_t)(stage * C::kStageSmem);
+#pragma unroll
+        for (int r = warp; r < 16; r += HKV) {
+            const int ph = r < t.count ? pt[x0 + r] : -1;
+            const bool ok = ph >= 0 && ph < p.s.NPG;
+            const uint8_t* src = p.meta8 + (size_t)(ok ? ph : 0) * HKV * C::kRowBytes;
+            const uint32_t d = dst + (uint32_t)(r * C::kRowBytes);
+#pragma unroll
+            for (int i = 0; i < C::kPageIters; ++i) {
+                const int j = lane + 32 * i;
+                if (C::kPageChunks % 32 == 0 || j < C::kPageChunks)
+                    cp_async_16(d + doff[i], src + 16 * j, ok ? 16u : 0u);
+            }
+        }
+    };
+
+    uint32_t qf[D / 8][NB][2];
+    int qexp[NB][2];
+    int cur_b = -1;
+    KeyRange kr;
+    const int g = warp;
+
+    auto process = [&](const TileInfo& t, int x0, int stage) {
+        const int b = t.unit;                               // walker over sequences
+        if (b != cur_b) {
+            cur_b = b;
+            load_q_frags<D, NB, true>(p, b, g, lane, qf, qexp);
+        }
+        const uint32_t tile =
+            ring_s + (uint32_t)(stage * C::kStageSmem + g * C::kTileSmem) + lm_off;
+        float acc[NB][4], acc2[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[nb][i] = acc2[nb][i] = 0.f;
+#pragma unroll
+        for (int kp = 0; kp < D / 16; ++kp) {
+            uint32_t m[4];
+            ldsm_x4(m, tile + 32 * kp);
+            const uint32_t a0[4] = {e4m3x2_to_f16x2(m[0]), e4m3x2_to_f16x2(m[1]),
+                                    e4m3x2_to_f16x2(m[0] >> 16), e4m3x2_to_f16x2(m[1] >> 16)};
+            const uint32_t a1[4] = {e4m3x2_to_f16x2(m[2]), e4m3x2_to_f16x2(m[3]),
+                                    e4m3x2_to_f16x2(m[2] >> 16), e4m3x2_to_f16x2(m[3] >> 16)};
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                mma_f16_16816(acc[nb], a0, qf[2 * kp][nb][0], qf[2 * kp][nb][1]);
+                mma_f16_16816(acc2[nb], a1, qf[2 * kp + 1][nb][0], qf[2 * kp + 1][nb][1]);
+            }
+        }
+        const uint8_t* rows = ring + stage * C::kStageSmem + g * C::kTileSmem;
+        const int e0 = *reinterpret_cast<const int*>(rows + gq * C::kRowBytes + 2 * D);
+        const int e8 = *reinterpret_cast<const int*>(rows + (gq + 8) * C::kRowBytes + 2 * D);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            acc[nb][0] = scale_pow2(acc[nb][0] + acc2[nb][0], e0 + qexp[nb][0]);
+            acc[nb][1] = scale_pow2(acc[nb][1] + acc2[nb][1], e0 + qexp[nb][1]);
+            acc[nb][2] = scale_pow2(acc[nb][2] + acc2[nb][2], e8 + qexp[nb][0]);
+            acc[nb][3] = scale_pow2(acc[nb][3] + acc2[nb][3], e8 + qexp[nb][1]);
+        }
+        int p0, p8;
+        const bool ok0 = row_ok(p, pt, x0, gq, t.count, p0);
+        const bool ok8 = row_ok(p, pt, x0, gq + 8, t.count, p8);
+        score_store<NB>(p, TileInfo{b * HKV + g, t.first, t.count}, acc, ok0, ok8, kr, lane);
+    };
+
+    // groups of up to 16 pages, walked by every thread alike; copies run
+    // kStages - 1 groups ahead, and thread 0 leaves each group's descriptor
+    // in shared memory for the barrier that makes its stage visible
+    walk.start(s, e);
+    auto issue_next = [&](int stage) -> bool {
+        TileInfo t;
+        if (!walk.next(t)) return false;
+        const int x0 = walk.x - t.count - s;                // slice index of page 0
+        if (tid == 0) desc[stage] = make_int4(t.unit, t.first, t.count, x0);
+        issue(t, x0, stage);
+        return true;
+    };
+    int pending = 0;
+#pragma unroll
+    for (int k = 0; k < C::kStages - 1; ++k) {
+        if (issue_next(k)) ++pending;
+        cp_async_commit();
+    }
+    for (int stage = 0; pending > 0; stage = stage + 1 == C::kStages ? 0 : stage + 1) {
+        cp_async_wait<C::kStages - 2>();    // this thread's copies of the stage landed
+        __syncthreads();                    // everyone's; and the previous stage is free
+        if (issue_next(stage == 0 ? C::kStages - 1 : stage - 1)) ++pending;
+        cp_async_commit();
+        const int4 d = desc[stage];
+        process(TileInfo{d.x, d.y, d.z}, d.w, stage);
+        --pending;
+    }
+    cp_async_wait<0>();
+    kr.flush(p, lane);
+}
+
 // ------------------------------------------------------------ launch
 // Raises a kernel's dynamic shared-memory limit to `bytes` unless done[dev]
 // (the caller's per-kernel record of the largest limit set on each device)
@@ -654,14 +849,40 @@ cudaError_t launch_ring(const ScoreParams& p, cudaStream_t st) {
 }
 
 // bf16 metadata: the direct path at D <= 128, the ring at D = 256; the fp8
-// copy: the ring.  Measured on B200: a 256k layer's scoring (D = 128, 262k
-// rows) took 28.5 us direct against 30.2 us in the ring, and 90 against
-// 100 us at four times the rows; the 64k layer (D = 256) took 37.4 us per
-// layer step with the ring against 39.6 us direct; the fp8 copy, 24.7 us in
-// the ring against 29.5 us direct.
+// copy: page-major at 4 or 8 kv-heads, else the ring.  Measured on B200: a
+// 256k layer's scoring (D = 128, 262k rows) took 28.5 us direct against
+// 30.2 us in the ring, and 90 against 100 us at four times the rows; the 64k
+// layer (D = 256) took 37.4 us per layer step with the ring against 39.6 us
+// direct; the fp8 copy, 24.7 us in the ring against 29.5 us direct, and one
+// 256k layer's fp8 scoring call after an L2 flush 27.8 us page-major (four
+// CTAs per SM) against 30.7 us in the ring.
+template <int D, int NB, int HKV>
+cudaError_t launch_pm(const ScoreParams& p, cudaStream_t st) {
+    using C = PmCfg<D, NB, HKV>;
+    auto kern = score_pm_kernel<D, NB, HKV>;
+    static size_t smem_set[64] = {0};
+    // kCtasPerSm CTAs per SM, or more when a CTA's share of the candidate
+    // pages would overflow kScorePtCap
+    const long long pages = (long long)p.s.B * p.s.MP;
+    long long grid = (long long)C::kCtasPerSm * device_sm_count();
+    const long long need = (pages + kScorePtCap - 1) / kScorePtCap;
+    if (need > grid) grid = need;
+    const size_t smem = C::smem_bytes(p.s.B, C::pt_cap(p.s.B, p.s.MP, (int)grid));
+    cudaError_t e = ensure_smem(kern, smem, smem_set);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(C::kThreads), smem, st, p);
+}
+
 template <int D, int NB>
 cudaError_t launch_score_d(const ScoreParams& p, cudaStream_t st) {
-    if (p.meta8) return launch_ring<D, NB, true>(p, st);
+    if (p.meta8) {
+        // whole pages of 4 or 8 kv-heads (not 8 at D = 256, whose stage
+        // would not fit twice, nor 8 with 16-head groups, which spills)
+        if (p.s.Hkv == 4) return launch_pm<D, NB, 4>(p, st);
+        if constexpr (D <= 128 && NB == 1)
+            if (p.s.Hkv == 8) return launch_pm<D, NB, 8>(p, st);
+        return launch_ring<D, NB, true>(p, st);
+    }
     if constexpr (D == 256) return launch_ring<D, NB, false>(p, st);
     else return launch_direct<D, NB>(p, st);
 }

@@ -109,6 +109,18 @@ def test_fp8_group_sizes_and_head_dims(G, D, cuda):
     check_fp8(Fp8Run(wl.make_case(w, cuda)))
 
 
+@pytest.mark.parametrize("Hkv,D,G", [(4, 64, 1), (4, 128, 8), (4, 128, 16), (4, 256, 2),
+                                     (4, 256, 16), (8, 64, 8), (8, 128, 1), (8, 128, 16)])
+def test_fp8_page_major_shapes(Hkv, D, G, cuda):
+    """Shapes whose fp8 scores come from the page-major kernel (4 or 8
+    kv-heads; 4 at D = 256): many ragged sequences, some without candidates,
+    so that CTA ranges start, end and change sequence inside 16-page groups."""
+    lens = (3000, 2049, 17, 800, 4096, 1, 1500, 2200)
+    w = wl.Workload("fp8_pm", B=len(lens), Hq=Hkv * G, Hkv=Hkv, D=D, seq_lens=lens, prefix=40,
+                    window=100, budget=480, seed=19)
+    check_fp8(Fp8Run(wl.make_case(w, cuda)))
+
+
 def test_fp8_copy_after_appends_matches_rebuild(cuda):
     """64 single-token appends through csa_meta_update_fp8: the fp8 copy is
     the oracle's from the final cache, bit for bit."""
