@@ -121,6 +121,41 @@ def test_fp8_page_major_shapes(Hkv, D, G, cuda):
     check_fp8(Fp8Run(wl.make_case(w, cuda)))
 
 
+@pytest.mark.parametrize("Hkv", [2, 4])
+def test_fp8_scores_with_subnormal_rows(Hkv, cuda):
+    """Keys whose channel 0 is about 256 and whose other channels lie within
+    2^-8: every fp8 row keeps exponent 0, so the small channels are E4M3
+    subnormals (below 2^-6).  Their share of a score is about 2^-9 of it,
+    far above the tolerance, so the scores match the oracle's fp8 definition
+    only if no stage of the kernel drops a subnormal (4 kv-heads: the
+    page-major kernel; 2: the ring)."""
+    w = wl.Workload("fp8_subnormal", B=2, Hq=4 * Hkv, Hkv=Hkv, D=128, seq_lens=(3000, 2049),
+                    prefix=40, window=100, budget=480, seed=23)
+    case = wl.make_case(w, cuda)
+    g = torch.Generator(device=cuda).manual_seed(29)
+    k = (torch.rand(case.k_cache.shape, generator=g, device=cuda) * 2 - 1) * 2.0 ** -8
+    sign = torch.randint(0, 2, case.k_cache.shape[:-1], generator=g, device=cuda) * 2 - 1
+    k[..., 0] = 256.0 * sign
+    case.k_cache.copy_(k.to(torch.bfloat16))
+    run = Fp8Run(case)
+    h = run.host()
+    assert_meta8_equal(run, h)
+    m8 = run.oracle_meta8(h)
+    # the small channels are E4M3 subnormals: exponent field 0, mantissa nonzero
+    used = np.concatenate([h["pt"][b, :-(-int(h["sl"][b]) // PS)] for b in range(w.B)])
+    body = m8[used][:, :, np.r_[1:w.D, w.D + 1:2 * w.D]]
+    assert ((body & 0x78) == 0).mean() > 0.9 and ((body & 0x07) != 0).mean() > 0.5
+    ref = oracle.scores_fp8(run.od, h["q"], m8, h["pt"], h["sl"], w.prefix, case.window)
+    lay = run.layer
+    sc = torch.full((run.d.B, run.d.Hkv, run.d.max_pages_per_seq), float("nan"),
+                    dtype=torch.float32, device=cuda)
+    csa.score_select_fp8(run.d, case.q, lay.meta8, case.page_table, case.seq_lens, w.prefix,
+                         case.window, run.budget, lay.sel, lay.n_sel, lay.ws, scores_out=sc)
+    torch.cuda.synchronize()
+    assert csa.device_status(lay.ws) == 0
+    assert_scores_close(sc, ref)
+
+
 def test_fp8_copy_after_appends_matches_rebuild(cuda):
     """64 single-token appends through csa_meta_update_fp8: the fp8 copy is
     the oracle's from the final cache, bit for bit."""
