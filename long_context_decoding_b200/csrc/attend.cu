@@ -26,6 +26,8 @@
 //     kernels before the scoring kernel (the token append among them) have
 //     finished.  They run while the scoring kernel ends and while the
 //     clusters select, when DRAM would otherwise idle.
+// Both roles end in one loop over the CTA's jobs (its units' item segments
+// and record slots), so that the page loop appears once in the kernel.
 // The combine kernel then merges each unit's records of both roles.
 #include "attend_core.cuh"
 #include "common.cuh"
@@ -65,6 +67,13 @@ __global__ void __cluster_dims__(kCl, 1, 1)
     using C = FusedCfg<D, NB>;
     using T = typename C::Tile;
     __shared__ ClShared sh;
+    // this CTA's work: per job a unit, its segment [a, b) of the items, the
+    // sequence length and the record slot (one attention call site for both
+    // roles keeps one copy of the page loop in the instruction stream)
+    __shared__ int job_u[kFusedUnits], job_a[kFusedUnits], job_b[kFusedUnits],
+        job_len[kFusedUnits];
+    __shared__ float* job_rec[kFusedUnits];
+    __shared__ int n_jobs;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // swizzled page buffers need 1024-byte alignment in the shared window
     uint8_t* stages = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -130,6 +139,26 @@ __global__ void __cluster_dims__(kCl, 1, 1)
                 if (uoff[u + 1] == uoff[u]) rr2[2 * u] = make_int2(0, -1);
         }
         if (s >= e) return;
+        // jobs: the units of the slice, items indexed from s
+        if (tid == 0) {
+            const int u_first = find_unit(uoff, units, s);
+            const int u_last = find_unit(uoff, units, e - 1);
+            int nj = 0;
+            for (int u = u_first; u <= u_last; ++u) {
+                const long long a = s > uoff[u] ? s : uoff[u];
+                const long long bnd = e < uoff[u + 1] ? e : uoff[u + 1];
+                if (a >= bnd) continue;
+                job_u[nj] = u;
+                job_a[nj] = (int)(a - s);
+                job_b[nj] = (int)(bnd - s);
+                job_len[nj] = ulen[u];
+                job_rec[nj] = p.partials + ((size_t)c0 + u) * rs;
+                ++nj;
+                const int first = cta_of(uoff[u], T0, n_cta);
+                if (c0 == first) rr2[2 * u] = make_int2(first, cta_of(uoff[u + 1] - 1, T0, n_cta));
+            }
+            n_jobs = nj;
+        }
         for (long long x = s + tid; x < e; x += kClThreads) {
             const int u = find_unit(uoff, units, x);
             const SeqGeom sg = seq_geom(ulen[u], p.prefix, p.window);
@@ -142,79 +171,74 @@ __global__ void __cluster_dims__(kCl, 1, 1)
             }
             items[x - s] = make_int2(phys, page * 4 + mask);
         }
+    } else {
+        // ----------------------------------------------- selection role
+        cg::cluster_group cl = cg::this_cluster();
+        const int rank = (int)cl.block_rank();
+        const int u = (int)blockIdx.x / kCl;
+        const int b = u / Hkv;
+        int L = p.seq_lens[b];
+        if (L < 0 || L > MP * kPage) L = 0;                  // flagged by the scoring kernel
+        const SeqGeom sg = seq_geom(L, p.prefix, p.window);
+        const int n = sg.c_hi - sg.c_lo;
+        const int kk = P.k_pages < n ? P.k_pages : n;
+        const int c_lo = sg.c_lo;
+        const int lo = kk * rank / kCl, hi = kk * (rank + 1) / kCl;   // this CTA's share
+        int32_t* out = P.sel + (size_t)u * p.s.max_sel;
+        if (tid < G * D / 64) {     // this unit's queries (a caller input) into L1
+            const uint16_t* qrow =
+                p.q + ((size_t)b * p.s.Hq + (size_t)(u % Hkv) * G) * D + tid * 64;
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(qrow));
+        }
+        pdl_wait();                 // the scores, and the previous readers of sel
+        pdl_launch_dependents();
+
+        if (kk == n) {              // every candidate fits the budget
+            for (int j = lo + tid; j < hi; j += kClThreads) share[j - lo] = c_lo + j;
+        } else if (kk > 0) {
+            uint32_t kmin, kmax;
+            key_range(P.keyrange[u], kmin, kmax);
+            // only shared-memory stores before the barrier (its release then
+            // waits for no global store); each CTA writes its share of the
+            // output list afterwards
+            cluster_select(cl, sh, P.scores_ws + (size_t)u * MP + c_lo, n, kk, kmin, kmax,
+                           [&](int pos, int i) {
+                               const int dst = ((pos + 1) * kCl + kk - 1) / kk - 1;
+                               int* d = cl.map_shared_rank(share, dst);
+                               d[pos - kk * dst / kCl] = c_lo + i;
+                           });
+            cluster_sync_all();     // every share is complete; no remote access after this
+        }
+        if (rank == 0 && tid == 0) {   // every CTA read the key range before the last barrier
+            P.n_sel[u] = kk;
+            P.keyrange[u] = make_uint2(0u, 0u);
+            rr2[2 * u + 1] = make_int2((kCl - 1) * u, (kCl - 1) * u + kCl - 1);   // slots 8u + r
+        }
         __syncthreads();
-        const int u_first = find_unit(uoff, units, s);
-        const int u_last = find_unit(uoff, units, e - 1);
-        for (int u = u_first; u <= u_last; ++u) {
-            const long long a = s > uoff[u] ? s : uoff[u];
-            const long long bnd = e < uoff[u + 1] ? e : uoff[u + 1];
-            if (a >= bnd) continue;
-            attend_unit<D, NB, C::kWarps, C::kHalves>(A, u, ulen[u], items, s, a, bnd, stages, ms,
-                                                     ls, p.partials + ((size_t)c0 + u) * rs);
-            const int first = cta_of(uoff[u], T0, n_cta);
-            if (c0 == first && tid == 0)
-                rr2[2 * u] = make_int2(first, cta_of(uoff[u + 1] - 1, T0, n_cta));
+        const int cnt = hi - lo;
+        for (int j = tid; j < cnt; j += kClThreads) {
+            const int page = share[j];
+            out[lo + j] = page;
+            int phys = p.page_table[(size_t)b * MP + page];
+            if (phys < 0 || phys >= p.s.NPG) {
+                latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
+                phys = -1;
+            }
+            items[j] = make_int2(phys, page * 4 + kMaskRest);
         }
-        return;
-    }
-
-    // ----------------------------------------------- selection role
-    cg::cluster_group cl = cg::this_cluster();
-    const int rank = (int)cl.block_rank();
-    const int u = (int)blockIdx.x / kCl;
-    const int b = u / Hkv;
-    int L = p.seq_lens[b];
-    if (L < 0 || L > MP * kPage) L = 0;                  // flagged by the scoring kernel
-    const SeqGeom sg = seq_geom(L, p.prefix, p.window);
-    const int n = sg.c_hi - sg.c_lo;
-    const int kk = P.k_pages < n ? P.k_pages : n;
-    const int c_lo = sg.c_lo;
-    const int lo = kk * rank / kCl, hi = kk * (rank + 1) / kCl;   // this CTA's share
-    int32_t* out = P.sel + (size_t)u * p.s.max_sel;
-    if (tid < G * D / 64) {     // this unit's queries (a caller input) into L1
-        const uint16_t* qrow = p.q + ((size_t)b * p.s.Hq + (size_t)(u % Hkv) * G) * D + tid * 64;
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(qrow));
-    }
-    pdl_wait();                 // the scores, and the previous readers of sel
-    pdl_launch_dependents();
-
-    if (kk == n) {              // every candidate fits the budget
-        for (int j = lo + tid; j < hi; j += kClThreads) share[j - lo] = c_lo + j;
-    } else if (kk > 0) {
-        uint32_t kmin, kmax;
-        key_range(P.keyrange[u], kmin, kmax);
-        // only shared-memory stores before the barrier (its release then
-        // waits for no global store); each CTA writes its share of the
-        // output list afterwards
-        cluster_select(cl, sh, P.scores_ws + (size_t)u * MP + c_lo, n, kk, kmin, kmax,
-                       [&](int pos, int i) {
-                           const int dst = ((pos + 1) * kCl + kk - 1) / kk - 1;
-                           int* d = cl.map_shared_rank(share, dst);
-                           d[pos - kk * dst / kCl] = c_lo + i;
-                       });
-        cluster_sync_all();     // every share is complete; no remote access after this
-    }
-    if (rank == 0 && tid == 0) {   // every CTA read the key range before the last barrier
-        P.n_sel[u] = kk;
-        P.keyrange[u] = make_uint2(0u, 0u);
-        rr2[2 * u + 1] = make_int2((kCl - 1) * u, (kCl - 1) * u + kCl - 1);   // slots 8u + r
+        if (tid == 0) {             // one job: the share (an empty one leaves an empty record)
+            job_u[0] = u;
+            job_a[0] = 0;
+            job_b[0] = cnt;
+            job_len[0] = L;
+            job_rec[0] = p.partials + p.phase_floats + ((size_t)kCl * u + rank) * rs;
+            n_jobs = 1;
+        }
     }
     __syncthreads();
-    const int cnt = hi - lo;
-    for (int j = tid; j < cnt; j += kClThreads) {
-        const int page = share[j];
-        out[lo + j] = page;
-        int phys = p.page_table[(size_t)b * MP + page];
-        if (phys < 0 || phys >= p.s.NPG) {
-            latch_flag(p.flags, CSA_DEVFLAG_BAD_PAGE_ID);
-            phys = -1;
-        }
-        items[j] = make_int2(phys, page * 4 + kMaskRest);
-    }
-    __syncthreads();
-    attend_unit<D, NB, C::kWarps, C::kHalves>(A, u, L, items, 0, 0, cnt, stages, ms, ls,
-                                             p.partials + p.phase_floats +
-                                                 ((size_t)kCl * u + rank) * rs);
+    for (int jb = 0; jb < n_jobs; ++jb)
+        attend_unit<D, NB, C::kWarps, C::kHalves>(A, job_u[jb], job_len[jb], items, 0, job_a[jb],
+                                                 job_b[jb], stages, ms, ls, job_rec[jb]);
 }
 
 template <int D, int NB>
