@@ -63,13 +63,13 @@ __device__ __forceinline__ uint32_t pos_part(uint32_t w) {   // max(q, 0) per bf
     return r;
 }
 
-// Two E4M3 values (bytes 0 and 1 of w) -> f16x2, exactly (hardware cvt).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
-    uint32_t h2;
-    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
-        : "=r"(h2)
+// Four E4M3 values (the bytes of w) -> two f16x2: bytes 0, 1 to lo and 2, 3
+// to hi, exactly (hardware cvt on each 16-bit half).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
         : "r"(w));
-    return h2;
 }
 
 // 2^e as a normal float, e clamped to [-126, 127] (built from its exponent bits).
@@ -565,10 +565,11 @@ score_ring_kernel(ScoreParams p) {
             for (int kp = 0; kp < D / 16; ++kp) {         // chunks 2kp and 2kp+1, one MMA each
                 uint32_t m[4];
                 ldsm_x4(m, tile + 32 * kp);
-                const uint32_t a0[4] = {e4m3x2_to_f16x2(m[0]), e4m3x2_to_f16x2(m[1]),
-                                        e4m3x2_to_f16x2(m[0] >> 16), e4m3x2_to_f16x2(m[1] >> 16)};
-                const uint32_t a1[4] = {e4m3x2_to_f16x2(m[2]), e4m3x2_to_f16x2(m[3]),
-                                        e4m3x2_to_f16x2(m[2] >> 16), e4m3x2_to_f16x2(m[3] >> 16)};
+                uint32_t a0[4], a1[4];
+                e4m3x4_to_f16x2x2(m[0], a0[0], a0[2]);
+                e4m3x4_to_f16x2x2(m[1], a0[1], a0[3]);
+                e4m3x4_to_f16x2x2(m[2], a1[0], a1[2]);
+                e4m3x4_to_f16x2x2(m[3], a1[1], a1[3]);
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb) {
                     mma_f16_16816(acc[nb], a0, qf[2 * kp][nb][0], qf[2 * kp][nb][1]);
@@ -744,10 +745,11 @@ __global__ void __launch_bounds__(PmCfg<D, NB, HKV>::kThreads, PmCfg<D, NB, HKV>
         for (int kp = 0; kp < D / 16; ++kp) {
             uint32_t m[4];
             ldsm_x4(m, tile + 32 * kp);
-            const uint32_t a0[4] = {e4m3x2_to_f16x2(m[0]), e4m3x2_to_f16x2(m[1]),
-                                    e4m3x2_to_f16x2(m[0] >> 16), e4m3x2_to_f16x2(m[1] >> 16)};
-            const uint32_t a1[4] = {e4m3x2_to_f16x2(m[2]), e4m3x2_to_f16x2(m[3]),
-                                    e4m3x2_to_f16x2(m[2] >> 16), e4m3x2_to_f16x2(m[3] >> 16)};
+            uint32_t a0[4], a1[4];
+            e4m3x4_to_f16x2x2(m[0], a0[0], a0[2]);
+            e4m3x4_to_f16x2x2(m[1], a0[1], a0[3]);
+            e4m3x4_to_f16x2x2(m[2], a1[0], a1[2]);
+            e4m3x4_to_f16x2x2(m[3], a1[1], a1[3]);
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
                 mma_f16_16816(acc[nb], a0, qf[2 * kp][nb][0], qf[2 * kp][nb][1]);
