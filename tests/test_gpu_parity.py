@@ -369,6 +369,16 @@ def test_one_call_many_units_edge_geometry(lens, P, W, budget, cuda):
     check_one_call(Run(wl.make_case(w, cuda)))
 
 
+@pytest.mark.parametrize("B,Hkv", [(8, 4), (16, 2), (11, 3)])
+def test_one_call_at_the_fused_unit_limit(B, Hkv, cuda):
+    """32 units (the most the single selection + attention launch serves:
+    an 8-CTA cluster per unit beside the prefix/window CTAs) and 33 (the
+    fewest that take the separate kernels): every unit against the oracle."""
+    w = small(B=B, Hq=8 * Hkv, Hkv=Hkv, D=128, lens=tuple(1500 + 97 * i for i in range(B)),
+              prefix=16, window=64, budget=256)
+    check_one_call(Run(wl.make_case(w, cuda)))
+
+
 def test_one_call_many_units_ctx64k_batch8(cuda):
     """Batch 8 x 8 kv-heads at 64k (64 units, D = 128), the benchmark's
     larger-batch shape: every unit against the oracle."""
