@@ -204,17 +204,25 @@ class Clocks:
             self.p.kill()
         self.f.flush()
         self.f.seek(0)
-        rows = [r.split(", ") for r in self.f.read().strip().splitlines() if r.count(",") >= 9]
+        text = self.f.read()
         os.unlink(self.f.name)
-        if not rows:
-            return None
-        busy = [r for r in rows if r[3].strip().isdigit() and int(r[3]) >= 50] or rows
-        mhz = [float(r[1]) for r in busy if r[1].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in busy for i in range(4) if r[6 + i].strip() == "Active"})
-        return {"sm_mhz": statistics.median(mhz) if mhz else None,
-                "sm_max_mhz": float(busy[0][2]) if busy[0][2].strip().isdigit() else None,
-                "reasons": reasons, "samples": len(busy)}
+        return clocks_summary(text)
+
+
+def clocks_summary(text: str):
+    """Median SM clock, the maximum clock and the throttle reasons seen, from
+    nvidia-smi CSV rows in the order of Clocks.Q (no header, no units); rows
+    with the GPU at least 50% busy only, when there are any."""
+    rows = [r.split(", ") for r in text.strip().splitlines() if r.count(",") >= 9]
+    if not rows:
+        return None
+    busy = [r for r in rows if r[3].strip().isdigit() and int(r[3]) >= 50] or rows
+    mhz = [float(r[1]) for r in busy if r[1].strip().replace(".", "").isdigit()]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in busy for i in range(4) if r[6 + i].strip() == "Active"})
+    return {"sm_mhz": statistics.median(mhz) if mhz else None,
+            "sm_max_mhz": float(busy[0][2]) if busy[0][2].strip().isdigit() else None,
+            "reasons": reasons, "samples": len(busy)}
 
 
 # ---------------------------------------------------------------- CPU oracle
