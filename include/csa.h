@@ -105,7 +105,9 @@ enum {
                                      not ascending, or n_sel out of range     */
     CSA_DEVFLAG_BAD_SEQ_LEN = 4,  /* seq_len < 0 or > 16 * max_pages_per_seq,
                                      or shorter than the appended chunk       */
-    CSA_DEVFLAG_TIMEOUT = 8       /* reserved: no kernel of this version waits */
+    CSA_DEVFLAG_TIMEOUT = 8       /* a kernel's bounded wait for its own copies
+                                     ran out (the fp8 scoring of 4 or 8
+                                     kv-heads): that call's results are void */
 };
 
 /* Problem shape, passed by host pointer to every call. */
