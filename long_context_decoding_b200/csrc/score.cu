@@ -684,14 +684,11 @@ score_ring_kernel(ScoreParams p) {
 template <int D, int NB, int HKV>
 struct PmCfg {
     static constexpr int kRowBytes = 2 * D + 16;             // one (page, kv-head) row
-    static constexpr int kRowChunks = kRowBytes / 16;
-    static constexpr int kPageChunks = HKV * kRowChunks;     // one page, every kv-head
     static constexpr int kPageBytes = HKV * kRowBytes;       // one page, every kv-head
     static constexpr int kSlot = kPageBytes + 16;            // a page's slot in a stage (odd chunks)
     static constexpr int kStageSmem = 16 * kSlot;
     static constexpr int kWarps = HKV;
     static constexpr int kThreads = 32 * kWarps;
-    static constexpr int kPageIters = (kPageChunks + 31) / 32;   // per lane and page
     // CTAs per SM: at 4 kv-heads and D <= 128, four (three stages each;
     // measured faster than two or three CTAs with deeper rings), three where
     // four would spill registers (16-head groups at D = 128); else two
