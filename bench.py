@@ -532,6 +532,7 @@ def run_ours(args, dist: Dist, base: wl.Workload):
         if not args.no_secondary and base.name == wl.CTX256K.name:
             line["ctx64k"] = secondary_64k(dev, dist)
             line["many_units"] = secondary_many_units(dev, dist, line)
+            line["context_parallel"] = secondary_context_parallel(dev, dist)
 
         # ---- sparse against dense over context length, and the cost model
         if not args.no_sweep and base.name == wl.CTX256K.name:
@@ -744,6 +745,70 @@ def secondary_many_units(dev, dist: Dist, line):
                     "pages during the selection) and combine as separate launches",
             "timing": "batches of 20 graph replays, each after a 256 MB L2 flush (read); the "
                       "flush time subtracted; median of 3 batches"}
+
+
+PEER_GBS = 770.0   # measured NVLink peer-copy bandwidth per direction on this hardware
+
+
+def secondary_context_parallel(dev, dist: Dist):
+    """Context parallelism emulated on one GPU: the 256k stack's first layer
+    (window 512, budget 1024) with every sequence's pages split over R = 2
+    and 4 ranks.  Each rank's kernels are timed as graph replays after an L2
+    flush, one rank after another: its local scoring, then its step after
+    the score exchange (the global selection from the gathered scores, its
+    share of the selection and its decode), then the merge after the partial
+    exchange.  The two all-gathers are not run (one GPU): their bytes per
+    rank are reported with the time they take at the measured peer
+    bandwidth, as a bound, not a measurement."""
+    from long_context_decoding_b200 import context_parallel as cp
+    from long_context_decoding_b200 import csa
+    w = replace(wl.CTX256K, layers=1)
+    c = wl.make_case(w, dev, layer=0)
+    d = csa.make_dims(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.num_pages, w.max_sel)
+    lay = csa.Layer(d, c.k_cache, c.v_cache, c.page_table, c.seq_lens, w.prefix, c.window,
+                    c.budget)
+    lay.rebuild_meta()
+    scrub = torch.ones(64 << 20, dtype=torch.float32, device=dev)   # 256 MB
+    sink = torch.zeros((), device=dev)
+
+    def flush():
+        torch.sum(scrub, dim=0, out=sink)
+
+    t_one = dist.max(graph_time(lambda: lay.step(c.q, fused=True), 20, 5, flush))
+    ref = lay.out.float().clone()
+    lens = [int(x) for x in c.seq_lens.cpu()]
+    res = {"workload": w.name + " layer 0", "single_gpu_us": 1e6 * t_one, "ranks": []}
+    for R in (2, 4):
+        plan = cp.plan_shards(w.max_pages, R, w.prefix, c.window, lens)
+        ops = [cp.CudaOps(plan, d, cp.shard_from_global(plan, r, c.k_cache, c.v_cache, lay.meta,
+                                                        c.page_table, lens),
+                          c.seq_lens, w.prefix, c.window, c.budget) for r in range(R)]
+        scores = [o.local_scores(c.q).clone() for o in ops]
+        parts = [tuple(x.clone() for x in o.attend(c.q, scores)) for o in ops]
+        out, _ = ops[0].merge([x[0] for x in parts], [x[1] for x in parts])
+        torch.cuda.synchronize()
+        err = float((out.float() - ref).abs().max())
+        t_sc = [dist.max(graph_time(lambda o=o: o.local_scores(c.q), 10, 3, flush)) for o in ops]
+        t_at = [dist.max(graph_time(lambda o=o: o.attend(c.q, scores), 10, 3, flush)) for o in ops]
+        t_mg = dist.max(graph_time(lambda: ops[0].merge([x[0] for x in parts],
+                                                        [x[1] for x in parts]), 10, 3, flush))
+        score_bytes = [4 * w.B * w.Hkv * (plan.hi(r) - plan.lo(r)) for r in range(R)]
+        part_bytes = w.B * w.Hq * (2 * w.D + 4)
+        recv = max(sum(score_bytes) - sb for sb in score_bytes) + (R - 1) * part_bytes
+        comp = max(a + b for a, b in zip(t_sc, t_at)) + t_mg
+        res["ranks"].append({
+            "R": R, "score_us": [1e6 * t for t in t_sc], "select_decode_us": [1e6 * t for t in t_at],
+            "merge_us": 1e6 * t_mg, "rank_kernels_us_max": 1e6 * comp,
+            "exchange_bytes_received_per_rank": recv,
+            "exchange_us_at_peer_bandwidth": 1e6 * recv / (PEER_GBS * 1e9),
+            "max_abs_diff_vs_single_gpu": err})
+        del ops
+        torch.cuda.empty_cache()
+    res["note"] = ("ranks emulated one after another on one GPU; the all-gathers are not run: "
+                   "exchange_us_at_peer_bandwidth is bytes / 770 GB/s, a bound")
+    del lay, c
+    torch.cuda.empty_cache()
+    return res
 
 
 def planted_recall(sel, nsel, planted):
